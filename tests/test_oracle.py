@@ -1,0 +1,287 @@
+"""Pins for the CPU oracle (runs without a GPU).
+
+Each test checks the oracle against something other than itself: the
+closed-form E4M3 bit formula, a brute-force argmin rounding, golden spot
+values with citations, a dense NumPy fp64 attention, and invariants that hold
+for any correct softmax attention (single token, identical keys, zero query,
+split-count and page-permutation invariance, LSE additivity, causal prefix
+reduction, scale folding).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import np_reference as npr
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "e4m3_spot.txt")
+
+
+# --------------------------------------------------------------------------- E4M3
+
+def test_e4m3_value_map_matches_bit_formula(oracle_lib):
+    codes = np.arange(256)
+    ref = npr.e4m3_values(codes)
+    got = np.array([oracle_lib.e4m3_value(c) for c in codes])
+    assert np.array_equal(np.isnan(ref), np.isnan(got))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ref[ok], got[ok])
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF])
+    assert got[0x7E] == 448.0 and got[0xFE] == -448.0
+    assert np.nanmax(np.abs(got)) == 448.0
+
+
+def _golden_rows():
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            rows.append((float(parts[0]), int(parts[1], 16), " ".join(parts[2:])))
+    return rows
+
+
+@pytest.mark.parametrize("x,code,note", _golden_rows())
+def test_e4m3_golden_spot_values(oracle_lib, x, code, note):
+    assert oracle_lib.e4m3_encode(x) == code, note
+    assert int(npr.e4m3_round(np.array([x]))[0]) == code, note
+
+
+ALL_BF16 = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+
+
+@pytest.mark.parametrize("scale", [1.0, 2.0 ** -3, 6.0 / 448.0, 1.0 / 3.0, 3.7 / 448.0, 4096.0])
+def test_quantize_exhaustive_bf16_against_bruteforce(oracle_lib, scale):
+    inv = np.float32(1.0) / np.float32(scale)
+    got = oracle_lib.quantize(ALL_BF16, float(inv))
+    x = (ALL_BF16.astype(np.uint32) << 16).view(np.float32)
+    with np.errstate(invalid="ignore"):
+        prod = (x * inv).astype(np.float32)  # one fp32 RN multiply
+    ref = np.concatenate([npr.e4m3_round(prod[i:i + 8192]) for i in range(0, prod.size, 8192)])
+    nan_in = np.isnan(prod)
+    assert np.all(got[nan_in] == 0x7F)
+    assert np.array_equal(got[~nan_in], ref[~nan_in])
+    # saturation: nothing finite becomes NaN
+    assert not np.any(((got & 0x7F) == 0x7F) & ~nan_in)
+
+
+def test_quantize_round_trip_all_finite_codes(oracle_lib):
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    for k in (-4, 0, 3):
+        scale = 2.0 ** k
+        vals = npr.e4m3_values(codes) * scale
+        bits = (vals.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        assert np.array_equal(npr.bf16_bits_to_f64(bits), vals)  # exact in bf16
+        got = oracle_lib.quantize(bits, float(np.float32(1.0) / np.float32(scale)))
+        assert np.array_equal(got, codes)
+
+
+def test_quantize_monotone(oracle_lib):
+    x = np.linspace(-600, 600, 20001).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    xv = npr.bf16_bits_to_f64(bits)
+    order = np.argsort(xv, kind="stable")
+    codes = oracle_lib.quantize(bits, 1.0)
+    vals = npr.e4m3_values(codes)[order]
+    assert np.all(np.diff(vals) >= 0)
+
+
+# --------------------------------------------------------------------------- attention helpers
+
+def _case(rng, B, q_len, H, lens, fp8, shuffle=True, kv_std=1.0, scale=0.05):
+    pages = [-(-L // 64) for L in lens]
+    npg = sum(pages) + 2
+    perm = rng.permutation(npg) if shuffle else np.arange(npg)
+    maxp = max(pages)
+    bt = np.full((B, maxp), perm[-1], dtype=np.int32)
+    off = 0
+    for b, n in enumerate(pages):
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    vals = (rng.standard_normal((npg, 64, 576)) * kv_std).astype(np.float32)
+    if fp8:
+        import oracle  # inputs only: the quantiser itself is pinned by the tests above
+        bits = (vals.view(np.uint32) >> 16).astype(np.uint16)
+        kv = oracle.quantize(bits, float(np.float32(1.0) / np.float32(scale)))
+        kv_scale = float(np.float32(scale))  # the API carries kv_scale as fp32
+    else:
+        kv = (vals.view(np.uint32) >> 16).astype(np.uint16)
+        kv_scale = 1.0
+    qn = (rng.standard_normal((B, q_len, H, 512)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    qr = (rng.standard_normal((B, q_len, H, 64)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return dict(q_nope=qn, q_rope=qr, kv_pages=kv, kv_scale=kv_scale, block_table=bt,
+                seq_lens=np.array(lens, dtype=np.int32), q_len=q_len, H=H,
+                softmax_scale=float(np.float32(1.0 / math.sqrt(192.0))))  # fp32 in the API
+
+
+def _all_rows(c):
+    return np.arange(len(c["seq_lens"]) * c["q_len"] * c["H"], dtype=np.int64)
+
+
+def _oracle_decode(oracle_lib, c, rows=None):
+    rows = _all_rows(c) if rows is None else rows
+    return oracle_lib.decode_rows(c["q_nope"], c["q_rope"], c["kv_pages"], c["kv_scale"],
+                                  c["block_table"], c["seq_lens"], c["q_len"], c["H"],
+                                  c["softmax_scale"], rows)
+
+
+# --------------------------------------------------------------------------- attention pins
+
+@pytest.mark.parametrize("fp8", [True, False])
+@pytest.mark.parametrize("B,q_len,H,lens", [
+    (1, 1, 1, [1]), (1, 1, 4, [5]), (2, 2, 2, [64, 70]), (1, 4, 3, [130]), (3, 1, 2, [8, 1, 200]),
+])
+def test_decode_matches_dense_numpy(oracle_lib, fp8, B, q_len, H, lens):
+    rng = np.random.default_rng(B * 100 + q_len * 10 + H + (7 if fp8 else 0))
+    c = _case(rng, B, q_len, H, lens, fp8)
+    o, lse = _oracle_decode(oracle_lib, c)
+    O, LSE = npr.attend(**c)
+    np.testing.assert_allclose(o, O.reshape(-1, 512), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(lse, LSE.reshape(-1), rtol=1e-11, atol=1e-12)
+
+
+def test_single_token_returns_its_value(oracle_lib):
+    rng = np.random.default_rng(1)
+    c = _case(rng, 1, 1, 3, [1], fp8=True)
+    o, lse = _oracle_decode(oracle_lib, c)
+    row = c["kv_pages"][c["block_table"][0, 0], 0]
+    v = npr.e4m3_values(row) * c["kv_scale"]
+    for h in range(3):
+        assert np.array_equal(o[h], v[:512])
+        q = np.concatenate([npr.bf16_bits_to_f64(c["q_nope"][0, 0, h]), npr.bf16_bits_to_f64(c["q_rope"][0, 0, h])])
+        assert lse[h] == pytest.approx(c["softmax_scale"] * float(q @ v), rel=1e-12)
+
+
+def test_identical_keys_give_mean_and_log_length(oracle_lib):
+    rng = np.random.default_rng(2)
+    c = _case(rng, 1, 1, 2, [150], fp8=False, shuffle=True)
+    row = c["kv_pages"][c["block_table"][0, 0], 0].copy()
+    c["kv_pages"][:, :, :] = row[None, None, :]
+    o, lse = _oracle_decode(oracle_lib, c)
+    v = npr.bf16_bits_to_f64(row)
+    for h in range(2):
+        np.testing.assert_allclose(o[h], v[:512], rtol=0, atol=1e-14)
+        q = np.concatenate([npr.bf16_bits_to_f64(c["q_nope"][0, 0, h]), npr.bf16_bits_to_f64(c["q_rope"][0, 0, h])])
+        s = c["softmax_scale"] * float(q @ v)
+        assert lse[h] == pytest.approx(s + math.log(150), rel=1e-12)
+
+
+def test_zero_query_gives_mean_of_values(oracle_lib):
+    rng = np.random.default_rng(3)
+    c = _case(rng, 1, 1, 1, [97], fp8=True)
+    c["q_nope"][:] = 0
+    c["q_rope"][:] = 0
+    o, lse = _oracle_decode(oracle_lib, c)
+    t = np.arange(97)
+    vals = npr.e4m3_values(c["kv_pages"][c["block_table"][0][t // 64], t % 64]) * c["kv_scale"]
+    np.testing.assert_allclose(o[0], vals[:, :512].mean(axis=0), rtol=1e-12, atol=1e-14)
+    assert lse[0] == pytest.approx(math.log(97), rel=1e-13)
+
+
+@pytest.mark.parametrize("S", [1, 2, 4, 7, 64])
+def test_split_count_invariance_and_lse_additivity(oracle_lib, S):
+    rng = np.random.default_rng(10 + S)
+    c = _case(rng, 2, 2, 2, [300, 1000], fp8=True)
+    rows = _all_rows(c)
+    o, lse = _oracle_decode(oracle_lib, c)
+    ns = np.full(2, S, dtype=np.int32)
+    po, pl = oracle_lib.partials_rows(c["q_nope"], c["q_rope"], c["kv_pages"], c["kv_scale"],
+                                      c["block_table"], c["seq_lens"], ns, S, c["q_len"], c["H"],
+                                      c["softmax_scale"], rows)
+    # LSE additivity: LSE(all) = logsumexp over splits, computed here in fp64
+    finite = np.isfinite(pl)
+    m = np.where(finite, pl, -np.inf).max(axis=1)
+    lse_sum = m + np.log(np.where(finite, np.exp(pl - m[:, None]), 0.0).sum(axis=1))
+    np.testing.assert_allclose(lse_sum, lse, rtol=1e-12)
+    # the merge (fp32 partials as the GPU stores them) reproduces the unsplit result
+    n_per_row = ns[(rows // (c["H"] * c["q_len"]))]
+    co, cl = oracle_lib.combine(po.astype(np.float32), pl.astype(np.float32), n_per_row)
+    np.testing.assert_allclose(co, o, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(cl, lse, rtol=1e-6)
+
+
+def test_split_range_partition(oracle_lib):
+    for L in (1, 63, 64, 65, 1000, 4096, 131072):
+        for S in (1, 2, 3, 7, 32, 64, 200):
+            vis = L
+            got = [oracle_lib.split_range(L, S, s, vis) for s in range(S)]
+            n_pages = -(-L // 64)
+            c = -(-n_pages // S)
+            pos = 0
+            for s, (t0, t1) in enumerate(got):
+                assert t0 == pos or t1 == t0
+                assert t0 % 64 == 0 or t1 == t0
+                assert t1 - t0 <= c * 64
+                pos = max(pos, t1)
+            assert pos == L
+            assert sum(t1 - t0 for t0, t1 in got) == L
+    # causal clip: a shorter visible length truncates the last non-empty split
+    assert oracle_lib.split_range(1000, 4, 3, 900) == (768, 900)
+    assert oracle_lib.split_range(1000, 4, 3, 700) == (700, 700)
+
+
+def test_page_permutation_invariance(oracle_lib):
+    rng = np.random.default_rng(4)
+    c = _case(rng, 2, 1, 2, [200, 130], fp8=True, shuffle=False)
+    o1, l1 = _oracle_decode(oracle_lib, c)
+    npg = c["kv_pages"].shape[0]
+    perm = rng.permutation(npg)
+    inv = np.argsort(perm)
+    c2 = dict(c)
+    c2["kv_pages"] = c["kv_pages"][perm]          # physical page p moves to slot inv[p]
+    c2["block_table"] = inv[c["block_table"]].astype(np.int32)
+    o2, l2 = _oracle_decode(oracle_lib, c2)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_causal_rows_equal_prefix_decode(oracle_lib):
+    rng = np.random.default_rng(5)
+    c = _case(rng, 1, 4, 2, [141], fp8=True)
+    o, lse = _oracle_decode(oracle_lib, c)
+    for q in range(4):
+        c1 = dict(c)
+        c1["q_len"] = 1
+        c1["q_nope"] = c["q_nope"][:, q:q + 1].copy()
+        c1["q_rope"] = c["q_rope"][:, q:q + 1].copy()
+        c1["seq_lens"] = np.array([141 - 3 + q], dtype=np.int32)
+        o1, l1 = _oracle_decode(oracle_lib, c1)
+        for h in range(2):
+            assert np.array_equal(o[q * 2 + h], o1[h])
+            assert lse[q * 2 + h] == l1[h]
+
+
+def test_fp8_scale_folding_equals_bf16_of_dequantised_values(oracle_lib):
+    rng = np.random.default_rng(6)
+    c = _case(rng, 1, 1, 2, [77], fp8=True, scale=0.125)
+    vals = npr.e4m3_values(c["kv_pages"]) * 0.125
+    vals = np.nan_to_num(vals, nan=0.0)
+    bits = (vals.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(npr.bf16_bits_to_f64(bits), vals)
+    o1, l1 = _oracle_decode(oracle_lib, c)
+    c2 = dict(c)
+    c2["kv_pages"] = bits
+    c2["kv_scale"] = 1.0
+    o2, l2 = _oracle_decode(oracle_lib, c2)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13)
+
+
+def test_combine_closed_forms(oracle_lib):
+    rng = np.random.default_rng(7)
+    po = rng.standard_normal((3, 4, 512)).astype(np.float32)
+    pl = np.array([[0.5, -1.0, -np.inf, -np.inf],
+                   [-np.inf, -np.inf, -np.inf, -np.inf],
+                   [2.0, 0, 0, 0]], dtype=np.float32)
+    ns = np.array([3, 4, 1], dtype=np.int32)
+    o, lse = oracle_lib.combine(po, pl, ns)
+    a, b = 0.5, -1.0
+    p64 = po.astype(np.float64)
+    want = (math.exp(a) * p64[0, 0] + math.exp(b) * p64[0, 1]) / (math.exp(a) + math.exp(b))
+    np.testing.assert_allclose(o[0], want, rtol=1e-12)
+    assert lse[0] == pytest.approx(math.log(math.exp(a) + math.exp(b)), rel=1e-12)
+    assert np.all(o[1] == 0) and lse[1] == -np.inf
+    np.testing.assert_allclose(o[2], po[2, 0].astype(np.float64), rtol=0, atol=0)
+    assert lse[2] == pytest.approx(2.0)
