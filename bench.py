@@ -1,0 +1,429 @@
+"""Benchmark: absorbed-MLA split-KV decode step on B200.
+
+A step is one pass of the decode hot path over one batch: mla_decode_partial
+(split-KV partial attention, steps A2-A8) followed by mla_combine (LSE merge,
+step A9) on one stream, inputs resident in HBM.  The FP8 cache itself is
+produced once per run by mla_quantize_fp8 (step A1), which is timed on its
+own and reported under "quantize".
+
+Default workload: batch 1, q_len 1, 64 heads, 128K context, FP8 E4M3 paged
+KV (page 64, shuffled block table), 64-way split.  The batch-16 workload (same
+shape, 32-way split) is measured in the same run and reported under
+"batch16".  L2 is flushed (a 256 MiB write) before every timed step, outside
+the timed events, so the 75.5 MB batch-1 cache is read from HBM.
+
+value = KV bytes read per step (sum_b L_b * 576) over all ranks / step time,
+in GB/s; ms_per_step is the device time of one step (max over ranks).
+With --gpus N > 1 every rank runs its own replica of the workload (the
+batch's requests are independent; no collective on the data path) and the
+timing is the max over ranks.
+
+--impl reference times the CPU oracle (the only reference implementation
+available) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode µs/step and KV-read HBM GB/s (% of peak) at 128K ctx, batch 1/16"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mla_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup_workload(name, device):
+    import torch
+    import mla_split_kv_absorbed_b200 as m
+    from mla_split_kv_absorbed_b200 import workloads as wl
+    w = wl.make(name, device=device)
+    if w.spec.kv_dtype == "fp8":
+        kv = torch.empty(w.kv_pool.shape, dtype=torch.uint8, device=device)
+        m.mla_quantize_fp8(w.kv_pool, kv, w.inv_scale)
+    else:
+        kv = w.kv_pool
+    torch.cuda.synchronize()
+    return w, kv
+
+
+def time_quantize(w, kv, reps=5):
+    """Step A1 over the whole pool: GB/s of (2 + 1) bytes per element."""
+    import torch
+    import mla_split_kv_absorbed_b200 as m
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    n = w.kv_pool.numel()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        m.mla_quantize_fp8(w.kv_pool, kv, w.inv_scale)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    t = min(times[1:]) if len(times) > 1 else times[0]
+    return {"elements": n, "us": t * 1e6, "gbs": 3.0 * n / t / 1e9}
+
+
+def run_steps(w, kv, steps, warmup, flush_bytes=256 << 20):
+    """Time `steps` decode steps (partial + combine) with an L2 flush before each.
+
+    Returns per-step total device times and per-step partial-kernel times (s)."""
+    import torch
+    import mla_split_kv_absorbed_b200 as m
+    stream = torch.cuda.current_stream()
+    part_o, part_lse = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
+    out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    out_lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
+    flush = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        m.mla_decode_partial(w.q_nope, w.q_rope, kv, w.kv_scale, w.block_table, w.seq_lens,
+                             w.num_splits, w.max_splits, w.softmax_scale, part_o, part_lse, err,
+                             stream)
+        if ev is not None:
+            ev[1].record(stream)
+        m.mla_combine(part_o, part_lse, w.num_splits, w.max_splits, out, out_lse, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    total = [e[0].elapsed_time(e[2]) * 1e-3 for e in evs]
+    partial = [e[0].elapsed_time(e[1]) * 1e-3 for e in evs]
+    return total, partial
+
+
+def run_e2e(w, kv, steps, warmup):
+    """Same step through the public API with host buffers: per step, pinned-host
+    -> device copies of the step's inputs (queries, seq_lens, num_splits,
+    block table), partial + combine, and device -> host copies of O and LSE.
+    The KV cache stays resident in HBM, as in serving."""
+    import torch
+    import mla_split_kv_absorbed_b200 as m
+    stream = torch.cuda.current_stream()
+    h_in = [t.cpu().pin_memory() for t in (w.q_nope, w.q_rope, w.seq_lens, w.num_splits, w.block_table)]
+    d_in = [torch.empty_like(t, device="cuda") for t in h_in]
+    part = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
+    out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    out_lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(out_lse.shape, dtype=out_lse.dtype).pin_memory()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = out.numel() * 2 + out_lse.numel() * 4
+
+    def step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        m.decode(d_in[0], d_in[1], kv, w.kv_scale, d_in[4], d_in[2], d_in[3], w.max_splits,
+                 w.softmax_scale, out=out, out_lse=out_lse, workspace=part)
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(out_lse, non_blocking=True)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    return statistics.median(times), h2d, d2h
+
+
+def cpu_baseline(w, kv_codes_host, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample: whole query rows of the
+    workload (all tokens of the row), as many as fit in about budget_s; the
+    projected full-step time gives the same GB/s metric."""
+    import numpy as np
+    import oracle
+    from mla_split_kv_absorbed_b200 import workloads as wl
+    qn, qr = wl.bf16_bits(w.q_nope), wl.bf16_bits(w.q_rope)
+    bt, sl = w.block_table.cpu().numpy(), w.seq_lens.cpu().numpy()
+    R = w.B * w.q_len * w.H
+    threads = oracle.num_threads()
+    rows_done, t_used, batch = 0, 0.0, threads
+    while t_used < budget_s and rows_done < R:
+        rows = np.arange(rows_done, min(R, rows_done + batch), dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.decode_rows(qn, qr, kv_codes_host, w.kv_scale, bt, sl, w.q_len, w.H, w.softmax_scale, rows)
+        t_used += time.perf_counter() - t0
+        rows_done += rows.size
+    t_step = t_used * R / rows_done
+    return {"value": w.kv_bytes / t_step / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows_done} of {R} query rows (all {int(sl.max())} tokens each), "
+                      f"{t_used:.1f} s, projected to a full step ({t_step:.1f} s)"}
+
+
+def host_codes(w, kv):
+    """FP8 codes for the oracle, produced by the oracle's own quantiser."""
+    import oracle
+    from mla_split_kv_absorbed_b200 import workloads as wl
+    if w.spec.kv_dtype == "fp8":
+        return oracle.quantize(wl.bf16_bits(w.kv_pool), w.inv_scale)
+    return wl.bf16_bits(w.kv_pool)
+
+
+def dist_setup():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="b1_128k_fp8")
+    ap.add_argument("--no-batch16", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import mla_split_kv_absorbed_b200 as m
+    ws, rank, local = dist_setup()
+    peak, peak_kind = load_peaks()
+
+    w, kv = setup_workload(args.workload, "cuda")
+    quant = time_quantize(w, kv) if w.spec.kv_dtype == "fp8" else None
+
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0 = time.perf_counter()
+        total, partial = run_steps(w, kv, args.steps, args.warmup)
+        wall = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    barrier(ws)
+    t_step = max_over_ranks(statistics.median(total), ws)
+    t_partial = max_over_ranks(statistics.median(partial), ws)
+    value = ws * w.kv_bytes / t_step / 1e9
+
+    e2e_t, h2d, d2h = run_e2e(w, kv, max(5, args.steps // 2), args.warmup)
+    e2e_t = max_over_ranks(e2e_t, ws)
+
+    extra = {}
+    if not args.no_batch16 and args.workload == "b1_128k_fp8":
+        w16, kv16 = setup_workload("b16_128k_fp8", "cuda")
+        tot16, par16 = run_steps(w16, kv16, max(5, args.steps // 2), args.warmup)
+        t16 = max_over_ranks(statistics.median(tot16), ws)
+        p16 = max_over_ranks(statistics.median(par16), ws)
+        extra["batch16"] = {"workload": "b16_128k_fp8", "us_per_step": t16 * 1e6,
+                            "kv_gbs": w16.kv_bytes / t16 / 1e9,
+                            "frac_of_peak": w16.kv_bytes / t16 / 1e9 / peak,
+                            "partial_us": p16 * 1e6, "partial_gbs": w16.kv_bytes / p16 / 1e9}
+        del kv16, w16
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, host_codes(w, kv))
+
+    achieved = w.kv_bytes / t_partial / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_step * 1e3,
+        "us_per_step": t_step * 1e6,
+        "frac_of_peak": w.kv_bytes / t_step / 1e9 / peak,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3" if w.spec.kv_dtype == "fp8" else "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "q_len": w.q_len, "H": w.H,
+                   "seq_len": int(w.seq_lens.max().item()), "num_splits": w.max_splits,
+                   "kv": w.spec.kv_dtype, "page": 64, "kv_bytes_per_step": w.kv_bytes,
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "decode_fp8_kernel" if w.spec.kv_dtype == "fp8" else "decode_bf16_kernel",
+                     "kernel_us": t_partial * 1e6, "peak_kind": peak_kind},
+        "e2e": {"value": ws * w.kv_bytes / e2e_t / 1e9, "unit": "GB/s", "us_per_step": e2e_t * 1e6,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "timed_wall_s": wall,
+    }
+    if quant is not None:
+        line["quantize"] = quant
+    line.update(extra)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def reference_arm(args):
+    """The oracle timed as the reference implementation (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from mla_split_kv_absorbed_b200 import workloads as wl
+    w = wl.make(args.workload, device="cpu")
+    codes = host_codes(w, None)
+    qn, qr = wl.bf16_bits(w.q_nope), wl.bf16_bits(w.q_rope)
+    bt, sl = w.block_table.numpy(), w.seq_lens.numpy()
+    R = w.B * w.q_len * w.H
+    threads = oracle.num_threads()
+    rows_per_step = threads
+    for _ in range(args.warmup):
+        oracle.decode_rows(qn, qr, codes, w.kv_scale, bt, sl, w.q_len, w.H, w.softmax_scale,
+                           np.arange(min(rows_per_step, R), dtype=np.int64))
+    times = []
+    for i in range(args.steps):
+        rows = (np.arange(rows_per_step, dtype=np.int64) + i * rows_per_step) % R
+        t0 = time.perf_counter()
+        oracle.decode_rows(qn, qr, codes, w.kv_scale, bt, sl, w.q_len, w.H, w.softmax_scale, rows)
+        times.append((time.perf_counter() - t0) * R / rows_per_step)
+    t_step = statistics.median(times)
+    value = w.kv_bytes / t_step / 1e9
+    sample = f"{rows_per_step} of {R} query rows per step (all tokens), projected to a full step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "q_len": w.q_len, "H": w.H,
+                   "seq_len": int(sl.max()), "num_splits": w.max_splits, "kv": w.spec.kv_dtype},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    main()

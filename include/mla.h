@@ -1,0 +1,150 @@
+/*
+ * mla.h — C ABI of the B200 (sm_100a) absorbed-MLA split-KV decode library.
+ *
+ * What the library computes (decode over a paged latent KV cache):
+ *   One KV row per token: 576 values = a 512-wide compressed latent (which is
+ *   also V) followed by a 64-wide decoupled RoPE key, stored as FP8 E4M3 codes
+ *   with one per-tensor scale, or as bf16.  For each query row (b, q, h):
+ *     s_t = softmax_scale * (q_nope . c_t[0:512] + q_rope . c_t[512:576])
+ *     O   = sum_t e^{s_t} c_t[0:512] / sum_t e^{s_t},  LSE = ln sum_t e^{s_t}
+ *   over the tokens the row sees.  q_nope is the already-absorbed 512-wide
+ *   query; absorption and the output up-projection belong to the caller.
+ *
+ * Sources: "SGLang & Miles ... Vera Rubin" article (arex-research.com),
+ * section "Kimi K3 的 MLA：更深的流水线、更快的 split-KV 归约":
+ *   - bullet "更快的 split-KV 归约": at low concurrency one request's KV is cut
+ *     across many CTAs, each producing a partial result, and a second kernel
+ *     merges the partials; the merge issues all partial loads first and then
+ *     accumulates from registers  -> mla_decode_partial + mla_combine;
+ *   - bullet "64 路 split-KV": batch-1 decode needs enough splits to occupy the
+ *     SMs  -> per-request num_splits, mla_choose_splits;
+ *   - bullet "原生 FP8 转换": KV/Q converted to FP8 with a saturating
+ *     conversion, overflow clamped to +-448 instead of NaN  -> mla_quantize_fp8.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless a name ends in _host.  The caller
+ *     owns all memory; the library allocates, frees and synchronises nothing.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is stream-ordered; the return value reports argument and
+ *     launch errors only.  Errors found by the GPU (bad page id, a wait that
+ *     timed out) are recorded in the caller's dev_error word, read after a
+ *     stream synchronisation.
+ *   - Arrays are dense, C order, as laid out below.  Device pointers must be
+ *     16-byte aligned (mla_quantize_fp8 also accepts unaligned pointers).
+ *   - Return 0 (MLA_OK) or one of the MLA_ERR_* codes; nothing is launched when
+ *     an argument is rejected.  No exceptions, no logging, no global state
+ *     other than a per-process cache of the device's SM count.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, out of range */
+  MLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. H*q_len not a multiple of 16) */
+  MLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed */
+  MLA_ERR_DEVICE = 4        /* reserved for callers that fold dev_error into a status */
+};
+
+enum {
+  MLA_KV_FP8_E4M3 = 0,      /* kv_pages holds E4M3 codes, value = code * kv_scale */
+  MLA_KV_BF16 = 1           /* kv_pages holds bf16 values, kv_scale must be 1 */
+};
+
+/* Bits the GPU ORs into *dev_error (zero it before the launch). */
+enum {
+  MLA_DEVERR_BAD_PAGE = 1,      /* block_table entry outside [0, num_pages); tile skipped */
+  MLA_DEVERR_BAD_SEQLEN = 2,    /* seq_len < q_len or above max_pages*64; request skipped */
+  MLA_DEVERR_TIMEOUT = 4,       /* a pipeline wait exceeded its time limit; CTA aborted */
+  MLA_DEVERR_BAD_SPLITS = 8,    /* num_splits[b] outside [1, max_splits]; request skipped */
+  MLA_DEVERR_SMEM_ALIGN = 16    /* dynamic shared memory base not 1 KiB aligned */
+};
+
+/* ---------------------------------------------------------------------------
+ * Step A1, prep: saturating FP8 conversion (article bullet "原生 FP8 转换").
+ *   y[i] = E4M3_RN_satfinite( fl32( float(x[i]) * inv_scale ) )
+ * x: n bf16 values (bit patterns), y: n E4M3 codes.  Exactly one fp32 multiply
+ * (round to nearest) then one E4M3 rounding, ties to even; |v| >= 448 and
+ * +-inf give +-448 (0x7E/0xFE), never NaN; NaN input gives an E4M3 NaN code.
+ * inv_scale is the caller's fp32 reciprocal of the dequantisation scale.
+ * n may be 0.  x and y may have any alignment (16-byte aligned is fastest).
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_quantize_fp8(const uint16_t* x_bf16, uint8_t* y_e4m3, int64_t n,
+                     float inv_scale, void* stream);
+
+/* Bytes of the split workspace: part_o (B*q_len*H*max_splits*512 fp32)
+ * followed by part_lse (B*q_len*H*max_splits fp32).  Returns 0 for invalid
+ * sizes.  A caller may carve both arrays from one allocation of this size
+ * (part_lse = part_o + B*q_len*H*max_splits*512). */
+MLA_API size_t mla_partial_workspace_bytes(int B, int q_len, int H, int max_splits);
+
+/* ---------------------------------------------------------------------------
+ * Steps A2-A8: split-KV partial attention (article bullet "更快的 split-KV 归约").
+ *
+ * q_nope     [B][q_len][H][512] bf16   absorbed query (latent part)
+ * q_rope     [B][q_len][H][64]  bf16   RoPE part of the query
+ * kv_pages   [num_pages][64][576]      E4M3 codes (kv_dtype 0) or bf16 (1)
+ * block_table[B][max_pages_per_req] int32: token t of request b is row t%64
+ *            of page block_table[b][t/64]
+ * seq_lens   [B] int32, tokens in the cache including the q_len new ones
+ *            (q_len <= seq_len <= max_pages_per_req*64)
+ * num_splits [B] int32 in [1, max_splits]
+ * Causality: query position q of request b sees tokens 0 .. seq_len-q_len+q.
+ * Split s of request b covers pages [s*c, min((s+1)*c, n)) with
+ * n = ceil(seq_len/64) and c = ceil(n/num_splits[b]).
+ * Outputs, for s < num_splits[b] (entries s >= num_splits[b] are not written):
+ *   part_o  [B][q_len][H][max_splits][512] fp32  O_s = sum_t w_t v_t / sum_t w_t
+ *   part_lse[B][q_len][H][max_splits]      fp32  LSE_s (natural log of the
+ *           scaled-score sum); an empty split gives O_s = 0, LSE_s = -inf.
+ * softmax_scale multiplies q.k; kv_scale (FP8 only) multiplies every code.
+ * Supported: H*q_len a multiple of 16, q_len in 1..4, H in 1..128,
+ * max_splits in 1..256.  dev_error may be NULL.
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope,
+                       const void* kv_pages, int kv_dtype, float kv_scale,
+                       int64_t num_pages, const int32_t* block_table,
+                       int max_pages_per_req, const int32_t* seq_lens,
+                       const int32_t* num_splits, int max_splits, int B, int q_len,
+                       int H, float softmax_scale, float* part_o, float* part_lse,
+                       int32_t* dev_error, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Step A9: the second kernel, LSE merge of the partials (same bullet): per row
+ *   M = max_s LSE_s, w_s = e^{LSE_s - M},
+ *   O = sum_s w_s O_s / sum_s w_s (rounded to bf16, nearest-even),
+ *   LSE = M + ln sum_s w_s   (fp32),
+ * over s < num_splits[b]; all splits empty gives O = 0, LSE = -inf.  Every
+ * partial load of a row is issued before the accumulation starts.
+ * out_bf16 [B][q_len][H][512], out_lse [B][q_len][H] (out_lse may be NULL).
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                int max_splits, int B, int q_len, int H, uint16_t* out_bf16,
+                float* out_lse, void* stream);
+
+/* Host helper (article bullet "64 路 split-KV"): per-request split counts that
+ * keep about two waves of CTAs on num_sms SMs, at least 16 pages per split,
+ * clamped to [1, max_splits].  seq_lens_host/out_host are HOST arrays of B. */
+MLA_API int mla_choose_splits(const int32_t* seq_lens_host, int B, int q_len, int H,
+                      int num_sms, int max_splits, int32_t* out_host);
+
+/* Static, human-readable name of a status code. */
+MLA_API const char* mla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

@@ -1,0 +1,200 @@
+"""Python binding of the B200 absorbed-MLA split-KV decode library.
+
+A thin ctypes layer over the C ABI in include/mla.h: it checks tensor dtypes,
+devices and shapes, passes raw device pointers and the current CUDA stream,
+and raises :class:`MlaError` on a non-zero status.  Every step of the decode
+runs in the library's CUDA kernels; there is no CPU or PyTorch fallback: the
+first call raises ImportError when the library has not been built.
+
+Entry points (same names as the C ABI):
+
+* ``mla_quantize_fp8(x_bf16, y_u8, inv_scale)`` — step A1, saturating E4M3.
+* ``mla_decode_partial(...)`` — steps A2-A8, per-split partial O and LSE.
+* ``mla_combine(...)`` — step A9, log-sum-exp merge into bf16 O and fp32 LSE.
+* ``mla_partial_workspace_bytes``, ``mla_choose_splits``, ``mla_status_string``.
+
+``decode(...)`` chains partial + combine with a caller-provided or freshly
+allocated workspace.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+
+MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_DEVICE = range(5)
+MLA_KV_FP8_E4M3, MLA_KV_BF16 = 0, 1
+DEVERR_BAD_PAGE, DEVERR_BAD_SEQLEN, DEVERR_TIMEOUT, DEVERR_BAD_SPLITS, DEVERR_SMEM_ALIGN = 1, 2, 4, 8, 16
+
+EXPORTS = ("mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
+           "mla_combine", "mla_choose_splits", "mla_status_string")
+
+
+class MlaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+_lib_handle = None
+
+
+def load():
+    """Load libmla_b200.so (raises ImportError if it has not been built)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load_lib()
+    return _lib_handle
+
+
+def _load_lib():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmla_b200.so is not built ({LIB_PATH}); run "
+                          "`python -m mla_split_kv_absorbed_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    lib.mla_quantize_fp8.argtypes = [P, P, i64, f32, P]
+    lib.mla_quantize_fp8.restype = i32
+    lib.mla_partial_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.mla_partial_workspace_bytes.restype = ctypes.c_size_t
+    lib.mla_decode_partial.argtypes = [P, P, P, i32, f32, i64, P, i32, P, P, i32, i32, i32, i32,
+                                       f32, P, P, P, P]
+    lib.mla_decode_partial.restype = i32
+    lib.mla_combine.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P]
+    lib.mla_combine.restype = i32
+    lib.mla_choose_splits.argtypes = [P, i32, i32, i32, i32, i32, P]
+    lib.mla_choose_splits.restype = i32
+    lib.mla_status_string.argtypes = [i32]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(load(), name)
+
+
+_lib = _LazyLib()
+
+
+def status_string(status: int) -> str:
+    return _lib.mla_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != MLA_OK:
+        raise MlaError(fn, status)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mla_quantize_fp8(x: torch.Tensor, y: torch.Tensor, inv_scale: float, stream=None):
+    """y (uint8 E4M3 codes) = saturating E4M3 of fl32(x * inv_scale); x bf16, same numel."""
+    if x.numel() != y.numel():
+        raise ValueError("x and y must have the same number of elements")
+    _check("mla_quantize_fp8", _lib.mla_quantize_fp8(
+        _dev(x, "x", torch.bfloat16), _dev(y, "y", torch.uint8), x.numel(), float(inv_scale),
+        _stream(stream)))
+    return y
+
+
+def mla_partial_workspace_bytes(B: int, q_len: int, H: int, max_splits: int) -> int:
+    return int(_lib.mla_partial_workspace_bytes(B, q_len, H, max_splits))
+
+
+def alloc_partials(B, q_len, H, max_splits, device="cuda"):
+    """(part_o [B][q_len][H][max_splits][512] fp32, part_lse [B][q_len][H][max_splits] fp32)."""
+    po = torch.empty((B, q_len, H, max_splits, 512), dtype=torch.float32, device=device)
+    pl = torch.empty((B, q_len, H, max_splits), dtype=torch.float32, device=device)
+    return po, pl
+
+
+def mla_decode_partial(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits,
+                       max_splits, softmax_scale, part_o, part_lse, dev_error=None, stream=None):
+    """Split-KV partial attention; kv_pages uint8 (E4M3) or bf16 [num_pages][64][576]."""
+    B, q_len, H, dl = q_nope.shape
+    if dl != 512 or tuple(q_rope.shape) != (B, q_len, H, 64):
+        raise ValueError("q_nope must be [B][q_len][H][512] and q_rope [B][q_len][H][64]")
+    if kv_pages.dim() != 3 or tuple(kv_pages.shape[1:]) != (64, 576):
+        raise ValueError("kv_pages must be [num_pages][64][576]")
+    if kv_pages.dtype == torch.uint8:
+        kv_dtype = MLA_KV_FP8_E4M3
+    elif kv_pages.dtype == torch.bfloat16:
+        kv_dtype = MLA_KV_BF16
+    else:
+        raise ValueError("kv_pages must be uint8 (E4M3 codes) or bfloat16")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B][max_pages]")
+    if part_o.numel() != B * q_len * H * max_splits * 512 or part_lse.numel() != B * q_len * H * max_splits:
+        raise ValueError("partial buffers have the wrong size")
+    _check("mla_decode_partial", _lib.mla_decode_partial(
+        _dev(q_nope, "q_nope", torch.bfloat16), _dev(q_rope, "q_rope", torch.bfloat16),
+        _dev(kv_pages, "kv_pages"), kv_dtype, float(kv_scale), kv_pages.shape[0],
+        _dev(block_table, "block_table", torch.int32), block_table.shape[1],
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(num_splits, "num_splits", torch.int32),
+        int(max_splits), B, q_len, H, float(softmax_scale),
+        _dev(part_o, "part_o", torch.float32), _dev(part_lse, "part_lse", torch.float32),
+        None if dev_error is None else _dev(dev_error, "dev_error", torch.int32), _stream(stream)))
+
+
+def mla_combine(part_o, part_lse, num_splits, max_splits, out, out_lse=None, stream=None):
+    """Merge partials into out (bf16 [B][q_len][H][512]) and out_lse (fp32 [B][q_len][H])."""
+    B, q_len, H, dl = out.shape
+    if dl != 512:
+        raise ValueError("out must be [B][q_len][H][512]")
+    _check("mla_combine", _lib.mla_combine(
+        _dev(part_o, "part_o", torch.float32), _dev(part_lse, "part_lse", torch.float32),
+        _dev(num_splits, "num_splits", torch.int32), int(max_splits), B, q_len, H,
+        _dev(out, "out", torch.bfloat16),
+        None if out_lse is None else _dev(out_lse, "out_lse", torch.float32), _stream(stream)))
+    return out
+
+
+def mla_choose_splits(seq_lens_host, q_len: int, H: int, num_sms: int, max_splits: int):
+    """Per-request split counts (host int32 tensor) for a host list/tensor of seq_lens."""
+    sl = torch.as_tensor(seq_lens_host, dtype=torch.int32).contiguous().cpu()
+    out = torch.empty_like(sl)
+    _check("mla_choose_splits", _lib.mla_choose_splits(
+        ctypes.c_void_p(sl.data_ptr()), sl.numel(), q_len, H, num_sms, max_splits,
+        ctypes.c_void_p(out.data_ptr())))
+    return out
+
+
+def mla_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def decode(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits, max_splits,
+           softmax_scale, out=None, out_lse=None, workspace=None, dev_error=None, stream=None):
+    """partial + combine; returns (out bf16 [B][q_len][H][512], out_lse fp32 [B][q_len][H])."""
+    B, q_len, H, _ = q_nope.shape
+    dev = q_nope.device
+    if workspace is None:
+        workspace = alloc_partials(B, q_len, H, max_splits, dev)
+    part_o, part_lse = workspace
+    if out is None:
+        out = torch.empty((B, q_len, H, 512), dtype=torch.bfloat16, device=dev)
+    if out_lse is None:
+        out_lse = torch.empty((B, q_len, H), dtype=torch.float32, device=dev)
+    mla_decode_partial(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits,
+                       max_splits, softmax_scale, part_o, part_lse, dev_error, stream)
+    mla_combine(part_o, part_lse, num_splits, max_splits, out, out_lse, stream)
+    return out, out_lse

@@ -1,0 +1,666 @@
+// Steps A2-A8 for an FP8 E4M3 latent cache: split-KV partial attention on
+// sm_100a tensor cores (tcgen05), fed by TMA.
+//
+// "SGLang & Miles ... Vera Rubin" article, section "Kimi K3 的 MLA":
+//  - bullet "更深的 MLA 流水线": long-context MLA decode waits on HBM KV
+//    reads; the fix is more reads in flight, i.e. a deep K/V shared-memory
+//    stage ring, with output bit-identical across pipeline depths;
+//  - bullet "更快的 split-KV 归约": one request's KV is cut across many CTAs,
+//    each writing a partial result (normalised O and its log-sum-exp) that a
+//    second kernel merges.
+//
+// One CTA = (query-row group g of up to 64 rows, split s, request b).  The
+// rows of a group are (q, h) pairs in [q_len][H] order.
+//
+// Tensor-core mapping (tokens as M): with at most 64 query rows per CTA,
+// using the rows as M would run the half-width M=64 UMMA shape and would need
+// a 64x512 fp32 O accumulator beside S, which does not fit TMEM.  Instead the
+// 128 tokens of a tile are M=128:
+//   S^T[t][n] = K[t][:] . Q[n][:]        A = K tile (K-major), B = Q (K-major)
+//   O^T[d][n] += V^T[d][t] . P[t][n]     A = V tile (MN-major), B = P (MN-major)
+// for d in four 128-wide blocks of the 512 latent dims.  V is the first 512
+// columns of the same resident tile that fed K, so every KV byte crosses HBM
+// once and shared memory once.
+//
+// Exact two-term FP8 operands: the cache is E4M3, and kind::f8f6f4 needs both
+// operands E4M3.  Q (bf16, 8 significant bits) is scaled per row by a power
+// of two and split as Q = Q_hi + Q_lo with Q_hi = E4M3(Q) and Q_lo =
+// E4M3(Q - Q_hi); this is exact for every element within 2^-10 of the row
+// maximum (smaller ones carry an absolute error below 2^-18 of the maximum).
+// B = [Q_hi ; Q_lo] is one N=128 operand, so S_hi and S_lo come out of one
+// MMA and the softmax adds them.  The softmax weights are scaled by 2^8,
+// p' = 2^(s - m + 8) in (0, 256], and split the same way, P = P_hi + P_lo:
+// about 8 significant bits (like bf16) for every p' >= 2^-2, and an absolute
+// error below 2^-10 (2^-18 of the row maximum) for smaller weights.  PV
+// accumulates both terms; the 2^8 cancels in O / l and is removed from LSE.
+//
+// Online softmax (log2 domain, scores pre-multiplied by log2 e): the running
+// max m per row only grows; when it grows, the O^T columns and the row sums
+// are rescaled by 2^(m_old - m_new) before the next PV accumulates.
+//
+// Warp roles (512 threads):
+//   warp 0        TMA producer: pages -> 64-byte-swizzled chunks
+//   warp 1        UMMA issuer (one thread) and TMEM owner
+//   warps 4-7     softmax, query columns 0-31   (thread = token row of S^T)
+//   warps 8-11    softmax, query columns 32-63
+//   warps 12-15   O^T rescaling between tiles, epilogue (thread = latent dim)
+//   warps 4-11    also convert Q to the split FP8 operand at the start
+// TMEM (512 columns): S^T buffers at 0 and 128 (S_hi 0-63 | S_lo 64-127),
+// O^T blocks at 256 + 64*j.
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "mla.h"
+#include "ptx.cuh"
+
+namespace mla {
+namespace fp8k {
+
+constexpr int kThreads = 512;
+constexpr int kRows = 64;           // query rows per CTA (UMMA N for PV)
+constexpr int kTile = 128;          // tokens per tile (UMMA M)
+constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
+constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
+constexpr int kRingPairs = 8;       // two tiles of latent dims in flight
+constexpr float kPShift = 8.0f;     // log2 of the factor carried by the softmax weights
+
+constexpr int kOffQ = 0;                                 // 9 chunks, rows hi 0-63 | lo 64-127
+constexpr int kOffRing = kOffQ + 9 * kChunk;             // 73728
+constexpr int kOffRope = kOffRing + kRingPairs * kPair;  // 204800
+constexpr int kOffPhi = kOffRope + kChunk;               // 212992
+constexpr int kOffPlo = kOffPhi + kChunk;                // 221184
+constexpr int kOffScratch = kOffPlo + kChunk;            // 229376
+constexpr int kSmemBytes = 232448;                       // 227 KiB
+
+// barrier indices
+constexpr int kBarNopeFull = 0;    // 8
+constexpr int kBarNopeEmpty = 8;   // 8
+constexpr int kBarRopeFull = 16;
+constexpr int kBarRopeEmpty = 17;
+constexpr int kBarSFull = 18;      // 2
+constexpr int kBarSEmpty = 20;     // 2
+constexpr int kBarPFull = 22;
+constexpr int kBarPEmpty = 23;
+constexpr int kBarOReady = 24;
+constexpr int kBarPvDone = 25;
+constexpr int kBarQReady = 26;
+constexpr int kBarAlphaFull = 27;
+constexpr int kBarDrain = 28;
+
+struct Scratch {
+  uint64_t bars[32];
+  uint32_t tmem_base;
+  int abort;
+  int pad[2];
+  float warp_max[2][4][32];  // per softmax group, per warp, per column; reused for row sums
+  float m_run[64];           // running max per column (log2 units)
+  float alpha[2][64];        // per tile parity: rescale factor per column
+  uint32_t changed[2][2];    // per tile parity, per column half: columns whose max grew
+  float c_head[64];          // per column: softmax_scale * kv_scale * log2(e) * 2^-e
+  float inv_l[64];           // per column: kv_scale / l  (0 when l == 0)
+  uint8_t qcol[64];          // per column: its query position q
+};
+static_assert(kOffScratch + sizeof(Scratch) <= kSmemBytes, "shared memory overflow");
+
+// 64-byte swizzle of a 64-byte-row layout: 16-byte unit u of row r lives at
+// unit u ^ ((r >> 1) & 3).  Matches the TMA 64B swizzle and the UMMA SW64
+// canonical layout when the atom base is 512-byte aligned.
+__device__ __forceinline__ uint32_t sw64(uint32_t row, uint32_t byte_in_row) {
+  return row * 64u + ((((byte_in_row >> 4) ^ ((row >> 1) & 3u)) << 4) | (byte_in_row & 15u));
+}
+
+__device__ __forceinline__ void set_error(int32_t* err, int bit) {
+  if (err != nullptr) atomicOr(err, bit);
+}
+
+// Convert 8 scaled fp32 query values into 8 hi and 8 lo E4M3 codes.
+__device__ __forceinline__ void split8(const float* x, uint2& hi, uint2& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t hc = cvt_e4m3x2(x[2 * k], x[2 * k + 1]);
+    const float2 back = half2_bits_to_float2(cvt_e4m3x2_to_f16x2((uint16_t)hc));
+    const uint32_t lc = cvt_e4m3x2(x[2 * k] - back.x, x[2 * k + 1] - back.y);
+    h[k] = hc;
+    l[k] = lc;
+  }
+  hi.x = h[0] | (h[1] << 16);
+  hi.y = h[2] | (h[3] << 16);
+  lo.x = l[0] | (l[1] << 16);
+  lo.y = l[2] | (l[3] << 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_fp8_kernel(const DecodeArgs args, const __grid_constant__ CUtensorMap kv_map) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  Scratch& sc = *reinterpret_cast<Scratch*>(smem + kOffScratch);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  const int g = blockIdx.x;
+  const int s = blockIdx.y;
+  const int b = blockIdx.z;
+  const int QH = args.q_len * args.H;
+
+  // ---------------------------------------------------------------- split range (step A2)
+  const int L = args.seq_lens[b];
+  const int S_b = args.num_splits[b];
+  if (S_b < 1 || S_b > args.max_splits) {
+    if (tid == 0 && s == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SPLITS);
+    return;
+  }
+  if (s >= S_b) return;
+  if (L < args.q_len || (int64_t)L > (int64_t)args.max_pages * 64) {
+    if (tid == 0 && s == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SEQLEN);
+    return;
+  }
+  const int n_pages = (L + 63) / 64;
+  const int cpages = (n_pages + S_b - 1) / S_b;
+  const int p0 = min(s * cpages, n_pages);
+  const int p1 = min(p0 + cpages, n_pages);
+  const int r0 = g * kRows;
+  const int rows_valid = min(kRows, QH - r0);
+  const int q_min = r0 / args.H;
+  const int q_max = (r0 + rows_valid - 1) / args.H;
+  const int vis_base = L - args.q_len + 1;  // visible length of q = 0
+  const int t0 = p0 * 64;
+  const int t1 = min(p1 * 64, vis_base + q_max);
+  const int t_all = min(t1, vis_base + q_min);  // every column sees every token < t_all
+  const int64_t row_base = (int64_t)b * QH + r0;
+
+  if (t1 <= t0) {  // empty split for every row of the group
+    for (int i = tid; i < rows_valid * 512; i += kThreads) {
+      const int n = i >> 9;
+      args.part_o[((row_base + n) * args.max_splits + s) * 512 + (i & 511)] = 0.0f;
+    }
+    if (tid < rows_valid) args.part_lse[(row_base + tid) * args.max_splits + s] = -INFINITY;
+    return;
+  }
+  const int T = (t1 - t0 + kTile - 1) / kTile;
+
+  // ---------------------------------------------------------------- setup
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (tid == 0) set_error(args.dev_error, MLA_DEVERR_SMEM_ALIGN);
+    return;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kRingPairs; ++i) {
+      mbar_init(&sc.bars[kBarNopeFull + i], 1);
+      mbar_init(&sc.bars[kBarNopeEmpty + i], 1);
+    }
+    mbar_init(&sc.bars[kBarRopeFull], 1);
+    mbar_init(&sc.bars[kBarRopeEmpty], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sc.bars[kBarSFull + i], 1);
+      mbar_init(&sc.bars[kBarSEmpty + i], 256);
+    }
+    mbar_init(&sc.bars[kBarPFull], 256);
+    mbar_init(&sc.bars[kBarPEmpty], 1);
+    mbar_init(&sc.bars[kBarOReady], 128);
+    mbar_init(&sc.bars[kBarPvDone], 1);
+    mbar_init(&sc.bars[kBarQReady], 8);
+    mbar_init(&sc.bars[kBarAlphaFull], 2);
+    mbar_init(&sc.bars[kBarDrain], 1);
+    sc.abort = 0;
+    fence_barrier_init();
+  }
+  if (tid < 64) {
+    sc.m_run[tid] = -INFINITY;
+    sc.qcol[tid] = (uint8_t)min((r0 + tid) / args.H, 255);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sc.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sc.tmem_base;
+  volatile int* abort_flag = &sc.abort;
+  uint64_t* bars = sc.bars;
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&kv_map);
+      const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
+      int last_nope_parity[kRingPairs];
+      bool armed[kRingPairs];
+      for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
+      int rope_armed_tiles = 0;
+      bool ok = true;
+      for (int i = 0; i < T && ok; ++i) {
+        const int tok0 = t0 + i * kTile;
+        const int pa = bt[p0 + 2 * i];
+        const bool want_b = tok0 + 64 < t1;
+        const int pb = want_b ? bt[p0 + 2 * i + 1] : 0;
+        bool la = (pa >= 0 && (int64_t)pa < args.num_pages);
+        bool lb = want_b && (pb >= 0 && (int64_t)pb < args.num_pages);
+        if (!la || (want_b && !lb)) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
+        const uint32_t bytes_chunk = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
+        for (int j = 0; j < 4; ++j) {
+          const int slot = (i & 1) * 4 + j;
+          if (i >= 2 && !(ok = mbar_wait(&bars[kBarNopeEmpty + slot], ((i - 2) >> 1) & 1, abort_flag)))
+            break;
+          uint64_t* full = &bars[kBarNopeFull + slot];
+          mbar_arrive_expect_tx(full, 2 * bytes_chunk);
+          armed[slot] = true;
+          last_nope_parity[slot] = (i >> 1) & 1;
+          uint8_t* dst = smem + kOffRing + slot * kPair;
+          for (int cc = 0; cc < 2; ++cc) {
+            const int chunk = 2 * j + cc;
+            if (la) tma_load_3d(dst + cc * kChunk, &kv_map, full, chunk * 64, 0, pa);
+            if (lb) tma_load_3d(dst + cc * kChunk + 4096, &kv_map, full, chunk * 64, 0, pb);
+          }
+        }
+        if (!ok) break;
+        if (i >= 1 && !(ok = mbar_wait(&bars[kBarRopeEmpty], (i - 1) & 1, abort_flag))) break;
+        uint64_t* rfull = &bars[kBarRopeFull];
+        mbar_arrive_expect_tx(rfull, bytes_chunk);
+        rope_armed_tiles = i + 1;
+        if (la) tma_load_3d(smem + kOffRope, &kv_map, rfull, 512, 0, pa);
+        if (lb) tma_load_3d(smem + kOffRope + 4096, &kv_map, rfull, 512, 0, pb);
+      }
+      // drain: every armed transaction has landed before the CTA may exit
+      const uint64_t t_start = globaltimer_ns();
+      for (int i = 0; i < kRingPairs; ++i)
+        if (armed[i])
+          while (!mbar_try_wait(&bars[kBarNopeFull + i], last_nope_parity[i]) &&
+                 globaltimer_ns() - t_start < kWaitLimitNs) {
+          }
+      if (rope_armed_tiles > 0)
+        while (!mbar_try_wait(&bars[kBarRopeFull], (rope_armed_tiles - 1) & 1) &&
+               globaltimer_ns() - t_start < kWaitLimitNs) {
+        }
+    }
+  } else if (warp == 1) {
+    // ============================================================ UMMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, 128, 128);  // E4M3 K-major x K-major, N=128
+      const uint32_t idesc_pv = instr_desc(0, 0, 1, 1, 128, 64);   // MN-major x MN-major, N=64
+      const uint32_t sQ = smem_u32(smem + kOffQ);
+      const uint32_t sRing = smem_u32(smem + kOffRing);
+      const uint32_t sRope = smem_u32(smem + kOffRope);
+      const uint32_t sPhi = smem_u32(smem + kOffPhi);
+      const uint32_t sPlo = smem_u32(smem + kOffPlo);
+      bool ok = mbar_wait(&bars[kBarQReady], 0, abort_flag);
+      tc_fence_after();
+      for (int i = 0; i <= T && ok; ++i) {
+        if (i < T) {
+          // ---------------- S^T(i) = K(i) . [Q_hi ; Q_lo]^T
+          const int sb = i & 1;
+          const uint32_t d_s = tmem + sb * 128;
+          if (i >= 2 && !(ok = mbar_wait(&bars[kBarSEmpty + sb], ((i - 2) >> 1) & 1, abort_flag)))
+            break;
+          tc_fence_after();
+          for (int j = 0; j < 4 && ok; ++j) {
+            const int slot = (i & 1) * 4 + j;
+            if (!(ok = mbar_wait(&bars[kBarNopeFull + slot], (i >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const uint32_t a_base = sRing + slot * kPair + cc * kChunk;
+              const uint32_t b_base = sQ + (2 * j + cc) * kChunk;
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk)
+                umma_f8(d_s, smem_desc(a_base + kk * 32, 16, 512, 4),
+                        smem_desc(b_base + kk * 32, 16, 512, 4), idesc_qk,
+                        (j | cc | kk) != 0 ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          if (!(ok = mbar_wait(&bars[kBarRopeFull], i & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            umma_f8(d_s, smem_desc(sRope + kk * 32, 16, 512, 4),
+                    smem_desc(sQ + 8 * kChunk + kk * 32, 16, 512, 4), idesc_qk, 1u);
+          umma_commit(&bars[kBarSFull + sb]);
+          umma_commit(&bars[kBarRopeEmpty]);
+        }
+        if (i >= 1) {
+          // ---------------- O^T += V(k)^T . (P_hi + P_lo)
+          const int k = i - 1;
+          if (!(ok = mbar_wait(&bars[kBarPFull], k & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&bars[kBarOReady], k & 1, abort_flag))) break;
+          tc_fence_after();
+          // the four O^T blocks are independent accumulators: issue them round-robin
+          // so that consecutive MMAs never wait on each other's accumulation
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int hl = 0; hl < 2; ++hl) {
+              const uint64_t bdesc = smem_desc((hl ? sPlo : sPhi) + kk * 2048, kChunk, 512, 4);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int slot = (k & 1) * 4 + j;
+                const uint64_t a = smem_desc(sRing + slot * kPair + kk * 2048, kChunk, 512, 4);
+                umma_f8(tmem + 256 + 64 * j, a, bdesc, idesc_pv,
+                        (k > 0 || kk > 0 || hl > 0) ? 1u : 0u);
+              }
+            }
+          }
+          umma_commit(&bars[kBarPEmpty]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) umma_commit(&bars[kBarNopeEmpty + (k & 1) * 4 + j]);
+          umma_commit(&bars[kBarPvDone]);
+        }
+      }
+      // drain: all issued MMAs complete before TMEM is released
+      umma_commit(&bars[kBarDrain]);
+      const uint64_t t_start = globaltimer_ns();
+      while (!mbar_try_wait(&bars[kBarDrain], 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ============================================================ Q split + softmax
+    const int wg = (warp - 4) >> 2;  // 0: columns 0-31, 1: columns 32-63
+    const int wq = warp & 3;         // TMEM lane quadrant
+    {
+      // ---- Q -> [Q_hi ; Q_lo] in K-major SW64 chunks, per-row power-of-two scale
+      const int pw = warp - 4;  // 0..7, rows pw, pw+8, ...
+      for (int n = pw; n < kRows; n += 8) {
+        const bool valid = n < rows_valid;
+        const uint16_t* qn = args.q_nope + (row_base + n) * 512;
+        const uint16_t* qr = args.q_rope + (row_base + n) * 64;
+        uint4 v[3];
+        int nch = 0;
+        int dim0[3];
+        if (valid) {
+          v[0] = *reinterpret_cast<const uint4*>(qn + lane * 8);
+          dim0[0] = lane * 8;
+          v[1] = *reinterpret_cast<const uint4*>(qn + 256 + lane * 8);
+          dim0[1] = 256 + lane * 8;
+          nch = 2;
+          if (lane < 8) {
+            v[2] = *reinterpret_cast<const uint4*>(qr + lane * 8);
+            dim0[2] = 512 + lane * 8;
+            nch = 3;
+          }
+        } else {
+          v[0] = v[1] = v[2] = make_uint4(0, 0, 0, 0);
+          dim0[0] = lane * 8;
+          dim0[1] = 256 + lane * 8;
+          dim0[2] = 512 + lane * 8;
+          nch = lane < 8 ? 3 : 2;
+        }
+        uint32_t amax_bits = 0;
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            amax_bits = max(amax_bits, (w[k] << 16) & 0x7FFFFFFFu);
+            amax_bits = max(amax_bits, w[k] & 0x7FFF0000u);
+          }
+        }
+        amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
+        const float amax = __uint_as_float(amax_bits);
+        int e = 0;
+        if (amax > 0.0f && amax_bits < 0x7F800000u) {
+          int E;
+          frexpf(amax, &E);
+          e = min(max(8 - E, -126), 126);
+        }
+        const float sc_up = __uint_as_float((uint32_t)(127 + e) << 23);
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+          float x[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            x[2 * k] = __uint_as_float(w[k] << 16) * sc_up;
+            x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u) * sc_up;
+          }
+          uint2 hi, lo;
+          split8(x, hi, lo);
+          const int chunk = dim0[c] >> 6;
+          const uint32_t bo = dim0[c] & 63;
+          uint8_t* base = smem + kOffQ + chunk * kChunk;
+          *reinterpret_cast<uint2*>(base + sw64(n, bo)) = hi;
+          *reinterpret_cast<uint2*>(base + sw64(64 + n, bo)) = lo;
+        }
+        if (lane == 0)
+          sc.c_head[n] = valid ? args.qk_scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23)
+                               : 0.0f;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarQReady]);
+      named_bar_sync(5, 256);  // c_head visible to both softmax groups
+    }
+
+    // ---- softmax over S^T: thread = token row r of the tile
+    const int r = wq * 32 + lane;
+    const int col0 = wg * 32;
+    const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+    float c_reg[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) c_reg[j] = sc.c_head[col0 + j];
+    float l_part[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) l_part[j] = 0.0f;
+    const int bar_id = 1 + wg;
+    bool ok = true;
+    for (int i = 0; i < T; ++i) {
+      const int sb = i & 1;
+      const int tok = t0 + i * kTile + r;
+      // one leader waits, the group follows after a named barrier (uniform outcome)
+      if (wq == 0 && lane == 0) mbar_wait(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag);
+      if (named_bar_or(bar_id, 128, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[32];
+      {
+        float hi[32], lo[32];
+        const uint32_t ts = t_lane + sb * 128 + col0;
+        tmem_ld16x2(ts, ts + 16, hi, hi + 16);
+        tmem_ld16x2(ts + 64, ts + 64 + 16, lo, lo + 16);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = (hi[j] + lo[j]) * c_reg[j];
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[kBarSEmpty + sb]);
+      // visibility mask (split end, causal limit per column, sequence end)
+      if (t0 + i * kTile + kTile > t_all) {
+        const int qq = tok - vis_base;  // token invisible to columns whose q <= qq
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (tok >= t1 || (qq >= 0 && (int)sc.qcol[col0 + j] <= qq)) sv[j] = -INFINITY;
+      }
+      // per-column tile max: warp redux, then across the 4 warps
+      float mine = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float wm = warp_max_f32(sv[j]);
+        mine = (lane == j) ? wm : mine;
+      }
+      sc.warp_max[wg][wq][lane] = mine;
+      named_bar_sync(bar_id, 128);
+      if (wq == 0) {
+        const int n = col0 + lane;
+        const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
+                               fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
+        const float m_old = sc.m_run[n];
+        const float m_new = fmaxf(m_old, tm);
+        const bool grew = m_new > m_old;
+        const float a = grew ? (m_old == -INFINITY ? 0.0f : exp2f(m_old - m_new)) : 1.0f;
+        sc.m_run[n] = m_new;
+        sc.alpha[i & 1][n] = a;
+        const uint32_t mask = __ballot_sync(0xffffffffu, grew);
+        if (lane == 0) sc.changed[i & 1][wg] = mask;
+      }
+      named_bar_sync(bar_id, 128);
+      if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull]);
+      // P buffer free (PV of the previous tile done)
+      if (i >= 1) {
+        if (wq == 0 && lane == 0) mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
+        if (named_bar_or(bar_id, 128, *abort_flag != 0)) {
+          ok = false;
+          break;
+        }
+      }
+      uint32_t phi[8], plo[8];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float m0 = sc.m_run[col0 + j], m1 = sc.m_run[col0 + j + 1];
+        const float a0 = sc.alpha[i & 1][col0 + j], a1 = sc.alpha[i & 1][col0 + j + 1];
+        // weights carry a 2^8 factor: p' = 2^(s - m + 8) in (0, 256], so that both
+        // E4M3 terms of every p' >= 2^-2 are normal numbers
+        const float p0v = (sv[j] == -INFINITY) ? 0.0f : exp2f(sv[j] - m0 + kPShift);
+        const float p1v = (sv[j + 1] == -INFINITY) ? 0.0f : exp2f(sv[j + 1] - m1 + kPShift);
+        l_part[j] = fmaf(l_part[j], a0, p0v);
+        l_part[j + 1] = fmaf(l_part[j + 1], a1, p1v);
+        const uint32_t hc = cvt_e4m3x2(p0v, p1v);
+        const float2 back = half2_bits_to_float2(cvt_e4m3x2_to_f16x2((uint16_t)hc));
+        const uint32_t lc = cvt_e4m3x2(p0v - back.x, p1v - back.y);
+        if ((j & 2) == 0) {
+          phi[j >> 2] = hc;
+          plo[j >> 2] = lc;
+        } else {
+          phi[j >> 2] |= hc << 16;
+          plo[j >> 2] |= lc << 16;
+        }
+      }
+      {
+        uint8_t* ph = smem + kOffPhi;
+        uint8_t* pl = smem + kOffPlo;
+        *reinterpret_cast<uint4*>(ph + sw64(r, col0)) = make_uint4(phi[0], phi[1], phi[2], phi[3]);
+        *reinterpret_cast<uint4*>(ph + sw64(r, col0 + 16)) = make_uint4(phi[4], phi[5], phi[6], phi[7]);
+        *reinterpret_cast<uint4*>(pl + sw64(r, col0)) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
+        *reinterpret_cast<uint4*>(pl + sw64(r, col0 + 16)) = make_uint4(plo[4], plo[5], plo[6], plo[7]);
+      }
+      if (tok >= t1) {
+        // rows past the visible range: clear their V bytes so 0 * garbage cannot be NaN
+        const int slot0 = (i & 1) * 4 + wg * 2;  // group 0 clears pairs 0-1, group 1 pairs 2-3
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + (slot0 + pp) * kPair + cc * kChunk + r * 64);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) row[u] = make_uint4(0, 0, 0, 0);
+          }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kBarPFull]);
+    }
+    // ---- row sums: reduce l_part over the 128 token rows of this group
+    {
+      float mine = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float v = l_part[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        mine = (lane == j) ? v : mine;
+      }
+      named_bar_sync(bar_id, 128);  // warp_max no longer read
+      sc.warp_max[wg][wq][lane] = mine;
+      named_bar_sync(bar_id, 128);
+      if (wq == 0) {
+        const int n = col0 + lane;
+        const float l = (sc.warp_max[wg][0][lane] + sc.warp_max[wg][1][lane]) +
+                        (sc.warp_max[wg][2][lane] + sc.warp_max[wg][3][lane]);
+        const bool nonempty = ok && l > 0.0f;
+        sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
+        if (n < rows_valid)
+          args.part_lse[(row_base + n) * args.max_splits + s] =
+              nonempty ? (sc.m_run[n] - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+    named_bar_sync(4, 384);  // inv_l ready for the epilogue
+  } else if (warp >= 12) {
+    // ============================================================ O^T rescale + epilogue
+    const int wq = warp & 3;
+    const int d_lane = wq * 32 + lane;  // latent dim within a 128-wide block
+    const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+    bool ok = true;
+    for (int i = 0; i < T; ++i) {
+      if (warp == 12 && lane == 0) {
+        mbar_wait(&bars[kBarAlphaFull], i & 1, abort_flag);
+        if (i >= 1) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
+      }
+      if (named_bar_or(3, 128, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (i >= 1) {
+        const uint32_t ch0 = sc.changed[i & 1][0], ch1 = sc.changed[i & 1][1];
+        if ((ch0 | ch1) != 0) {
+#pragma unroll 1
+          for (int grp = 0; grp < 4; ++grp) {
+            const uint32_t bits = ((grp < 2 ? ch0 : ch1) >> ((grp & 1) * 16)) & 0xFFFFu;
+            if (bits == 0) continue;
+            float a[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) a[c] = sc.alpha[i & 1][grp * 16 + c];
+#pragma unroll 1
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t ta = t_lane + 256 + 64 * j + 16 * grp;
+              float v[16];
+              tmem_ld16(ta, v);
+#pragma unroll
+              for (int c = 0; c < 16; ++c) v[c] *= a[c];
+              tmem_st16(ta, v);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[kBarOReady]);
+    }
+    if (ok && warp == 12 && lane == 0) mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
+    const bool bad = named_bar_or(3, 128, !ok || *abort_flag != 0);
+    named_bar_sync(4, 384);
+    if (!bad) {
+      tc_fence_after();
+      float* po = args.part_o + (row_base * args.max_splits + s) * 512;
+      const int64_t row_stride = (int64_t)args.max_splits * 512;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll 1
+        for (int grp = 0; grp < 4; ++grp) {
+          float v[16];
+          tmem_ld16(t_lane + 256 + 64 * j + 16 * grp, v);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int n = grp * 16 + c;
+            if (n < rows_valid) po[n * row_stride + 128 * j + d_lane] = v[c] * sc.inv_l[n];
+          }
+        }
+      }
+    }
+  }
+  // warps 2-3 and idle lanes fall through
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && tid == 0) set_error(args.dev_error, MLA_DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fp8k
+
+cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(fp8k::decode_fp8_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         fp8k::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int groups = (a.q_len * a.H + fp8k::kRows - 1) / fp8k::kRows;
+  dim3 grid(groups, a.max_splits, a.B);
+  fp8k::decode_fp8_kernel<<<grid, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

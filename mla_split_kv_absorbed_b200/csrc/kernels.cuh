@@ -1,0 +1,45 @@
+// Internal launcher declarations shared by the kernel files and the C ABI.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mla {
+
+cudaError_t launch_quantize_fp8(const uint16_t* x, uint8_t* y, int64_t n, float inv_scale,
+                                int num_sms, cudaStream_t stream);
+
+cudaError_t launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                           int max_splits, int B, int q_len, int H, uint16_t* out, float* out_lse,
+                           cudaStream_t stream);
+
+// Arguments of the split-KV partial kernels (device pointers; see mla.h).
+struct DecodeArgs {
+  const uint16_t* q_nope;
+  const uint16_t* q_rope;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const int32_t* num_splits;
+  float* part_o;
+  float* part_lse;
+  int32_t* dev_error;
+  int64_t num_pages;
+  int max_pages;
+  int max_splits;
+  int B;
+  int q_len;
+  int H;
+  float qk_scale_log2;  // softmax_scale * kv_scale * log2(e)
+  float kv_scale;
+};
+
+// FP8 E4M3 cache: kv_map is a 3-D tiled TMA map over kv_pages viewed as
+// [num_pages][64][576] bytes, box {64 B, 64 rows, 1 page}, 64-byte swizzle.
+cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cudaStream_t stream);
+
+// bf16 cache: kv_map over [num_pages][64][576] bf16, box {64 elems, 64 rows,
+// 1 page}, 128-byte swizzle.
+cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap& kv_map,
+                               cudaStream_t stream);
+
+}  // namespace mla

@@ -1,0 +1,193 @@
+// C ABI of the library (declarations and contracts in include/mla.h):
+// argument validation, TMA descriptor encoding and kernel launches.  Nothing
+// here allocates, frees or synchronises; every launch goes to the caller's
+// stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.cuh"
+#include "mla.h"
+
+namespace {
+
+constexpr int kPage = 64;
+constexpr int kRow = 576;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms_cached() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return 148;
+    sms = v;
+  }
+  return sms;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// TMA map over kv_pages viewed as [num_pages][64][576] elements with a box of
+// {64 elements, 64 rows, 1 page}: 64 B rows (64-byte swizzle) for E4M3,
+// 128 B rows (128-byte swizzle) for bf16.
+int make_kv_map(CUtensorMap* map, const void* kv_pages, int kv_dtype, int64_t num_pages) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return MLA_ERR_CUDA;
+  const cuuint64_t esz = kv_dtype == MLA_KV_FP8_E4M3 ? 1 : 2;
+  const cuuint64_t dims[3] = {(cuuint64_t)kRow, (cuuint64_t)kPage, (cuuint64_t)num_pages};
+  const cuuint64_t strides[2] = {kRow * esz, (cuuint64_t)kPage * kRow * esz};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map,
+                        kv_dtype == MLA_KV_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        3, const_cast<void*>(kv_pages), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        kv_dtype == MLA_KV_FP8_E4M3 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int mla_quantize_fp8(const uint16_t* x_bf16, uint8_t* y_e4m3, int64_t n, float inv_scale,
+                     void* stream) {
+  if (n < 0) return MLA_ERR_INVALID_ARG;
+  if (n == 0) return MLA_OK;
+  if (x_bf16 == nullptr || y_e4m3 == nullptr) return MLA_ERR_INVALID_ARG;
+  return status_of(mla::launch_quantize_fp8(x_bf16, y_e4m3, n, inv_scale, num_sms_cached(),
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_partial_workspace_bytes(int B, int q_len, int H, int max_splits) {
+  if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return 0;
+  const size_t rows = (size_t)B * q_len * H * max_splits;
+  return rows * 512 * sizeof(float) + rows * sizeof(float);
+}
+
+int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_pages,
+                       int kv_dtype, float kv_scale, int64_t num_pages,
+                       const int32_t* block_table, int max_pages_per_req,
+                       const int32_t* seq_lens, const int32_t* num_splits, int max_splits, int B,
+                       int q_len, int H, float softmax_scale, float* part_o, float* part_lse,
+                       int32_t* dev_error, void* stream) {
+  if (q_nope == nullptr || q_rope == nullptr || kv_pages == nullptr || block_table == nullptr ||
+      seq_lens == nullptr || num_splits == nullptr || part_o == nullptr || part_lse == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(kv_pages) || !aligned16(part_o))
+    return MLA_ERR_INVALID_ARG;
+  if (B <= 0 || q_len <= 0 || H <= 0 || num_pages <= 0 || max_pages_per_req <= 0 ||
+      max_splits <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (num_pages > 0x7FFFFFFFll || (int64_t)max_pages_per_req * kPage > 0x7FFFFFFFll)
+    return MLA_ERR_INVALID_ARG;
+  if (kv_dtype != MLA_KV_FP8_E4M3 && kv_dtype != MLA_KV_BF16) return MLA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale) || !(kv_scale == kv_scale) || kv_scale <= 0.0f)
+    return MLA_ERR_INVALID_ARG;
+  if (kv_dtype == MLA_KV_BF16 && kv_scale != 1.0f) return MLA_ERR_INVALID_ARG;
+  if (q_len > 4 || H > 128 || max_splits > 256 || B > 65535 || (q_len * H) % 16 != 0)
+    return MLA_ERR_UNSUPPORTED;
+
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  int st = make_kv_map(&map, kv_pages, kv_dtype, num_pages);
+  if (st != MLA_OK) return st;
+
+  mla::DecodeArgs a;
+  a.q_nope = q_nope;
+  a.q_rope = q_rope;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.num_splits = num_splits;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.dev_error = dev_error;
+  a.num_pages = num_pages;
+  a.max_pages = max_pages_per_req;
+  a.max_splits = max_splits;
+  a.B = B;
+  a.q_len = q_len;
+  a.H = H;
+  a.qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
+  a.kv_scale = kv_scale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, s)
+                                               : mla::launch_decode_bf16(a, map, s));
+}
+
+int mla_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                int max_splits, int B, int q_len, int H, uint16_t* out_bf16, float* out_lse,
+                void* stream) {
+  if (part_o == nullptr || part_lse == nullptr || num_splits == nullptr || out_bf16 == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return MLA_ERR_INVALID_ARG;
+  if (max_splits > 256 || q_len > 4 || H > 128) return MLA_ERR_UNSUPPORTED;
+  return status_of(mla::launch_combine(part_o, part_lse, num_splits, max_splits, B, q_len, H,
+                                       out_bf16, out_lse, static_cast<cudaStream_t>(stream)));
+}
+
+int mla_choose_splits(const int32_t* seq_lens_host, int B, int q_len, int H, int num_sms,
+                      int max_splits, int32_t* out_host) {
+  if (seq_lens_host == nullptr || out_host == nullptr || B <= 0 || q_len <= 0 || H <= 0 ||
+      num_sms <= 0 || max_splits <= 0)
+    return MLA_ERR_INVALID_ARG;
+  const int groups = (q_len * H + 63) / 64;
+  int64_t total_pages = 0;
+  for (int b = 0; b < B; ++b) {
+    if (seq_lens_host[b] < q_len) return MLA_ERR_INVALID_ARG;
+    total_pages += (seq_lens_host[b] + kPage - 1) / kPage;
+  }
+  // about two waves of (request, split, row-group) CTAs, at least 16 pages each
+  const int64_t target_ctas = 2 * (int64_t)num_sms;
+  int64_t pages_per_split = (total_pages * groups + target_ctas - 1) / target_ctas;
+  if (pages_per_split < 16) pages_per_split = 16;
+  for (int b = 0; b < B; ++b) {
+    const int64_t pages = (seq_lens_host[b] + kPage - 1) / kPage;
+    int64_t sp = (pages + pages_per_split - 1) / pages_per_split;
+    if (sp < 1) sp = 1;
+    if (sp > max_splits) sp = max_splits;
+    out_host[b] = (int32_t)sp;
+  }
+  return MLA_OK;
+}
+
+const char* mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE: return "MLA_ERR_DEVICE";
+    default: return "MLA_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"
