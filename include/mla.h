@@ -56,7 +56,8 @@ enum {
   MLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, out of range */
   MLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. H*q_len not a multiple of 16) */
   MLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed */
-  MLA_ERR_DEVICE = 4        /* reserved for callers that fold dev_error into a status */
+  MLA_ERR_DEVICE = 4,       /* reserved for callers that fold dev_error into a status */
+  MLA_ERR_SCRATCH_LIMIT = 5 /* mla_decode_noalloc: problem larger than its fixed scratch */
 };
 
 enum {
@@ -133,6 +134,36 @@ MLA_API int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope,
 MLA_API int mla_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
                 int max_splits, int B, int q_len, int H, uint16_t* out_bf16,
                 float* out_lse, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Allocation-free decode (steps A2-A9 in one call).  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory (a plugin whose host owns the whole device memory pool and
+ * offers no allocator, a latency-critical loop that must not call cudaMalloc
+ * because it may synchronise the device).  Arguments and outputs are those of
+ * mla_decode_partial followed by mla_combine, minus the workspace: the split
+ * partials live in a file-scope device array inside the library, and the
+ * library allocates nothing (no cudaMalloc, no cudaFree).
+ *   - Limit: B*q_len*H*max_splits <= 8192 (row, split) pairs, e.g. batch 1 x
+ *     64 heads x 128 splits; larger problems return MLA_ERR_SCRATCH_LIMIT and
+ *     launch nothing.  Every GPU on which the library is loaded holds that
+ *     array (8192*513 fp32, about 16 MiB) until the process exits.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress); make that first call before
+ *     any stream capture.  Later calls reuse the address.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents.  Each call writes every entry it reads, so nothing needs to
+ *     start at zero, but calls that overlap on the GPU (different streams,
+ *     host threads) race on it: order them on one stream.
+ *   - If dev_error reports an error the outputs are undefined.
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_decode_noalloc(const uint16_t* q_nope, const uint16_t* q_rope,
+                               const void* kv_pages, int kv_dtype, float kv_scale,
+                               int64_t num_pages, const int32_t* block_table,
+                               int max_pages_per_req, const int32_t* seq_lens,
+                               const int32_t* num_splits, int max_splits, int B, int q_len,
+                               int H, float softmax_scale, uint16_t* out_bf16, float* out_lse,
+                               int32_t* dev_error, void* stream);
 
 /* Host helper (article bullet "64 路 split-KV"): per-request split counts that
  * keep about two waves of CTAs on num_sms SMs, at least 16 pages per split,

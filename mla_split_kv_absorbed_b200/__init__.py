@@ -27,6 +27,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_DEVICE = range(5)
+MLA_ERR_SCRATCH_LIMIT = 5
 MLA_KV_FP8_E4M3, MLA_KV_BF16 = 0, 1
 DEVERR_BAD_PAGE, DEVERR_BAD_SEQLEN, DEVERR_TIMEOUT, DEVERR_BAD_SPLITS, DEVERR_SMEM_ALIGN = 1, 2, 4, 8, 16
 

@@ -186,6 +186,7 @@ const char* mla_status_string(int status) {
     case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
     case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
     case MLA_ERR_DEVICE: return "MLA_ERR_DEVICE";
+    case MLA_ERR_SCRATCH_LIMIT: return "MLA_ERR_SCRATCH_LIMIT";
     default: return "MLA_ERR_UNKNOWN";
   }
 }
