@@ -24,23 +24,27 @@
 //
 // Exact two-term FP8 operands: the cache is E4M3, and kind::f8f6f4 needs both
 // operands E4M3.  Q (bf16, 8 significant bits) is scaled per row by a power
-// of two and split as Q = Q_hi + Q_lo with Q_hi = E4M3(Q) and Q_lo =
-// E4M3(Q - Q_hi); this is exact for every element within 2^-10 of the row
-// maximum (smaller ones carry an absolute error below 2^-18 of the maximum).
-// B = [Q_hi ; Q_lo] is one N=128 operand, so S_hi and S_lo come out of one
-// MMA and the softmax adds them.  The softmax weights are scaled by 2^8,
-// p' = 2^(s - m + 8) in (0, 256], and split the same way, P = P_hi + P_lo:
-// about 8 significant bits (like bf16) for every p' >= 2^-2, and an absolute
-// error below 2^-10 (2^-18 of the row maximum) for smaller weights.  PV
-// accumulates both terms; the 2^8 cancels in O / l and is removed from LSE.
+// of two and split as Q = Q_hi + Q_lo with Q_hi = Q rounded to 4 significant
+// bits and Q_lo = E4M3(Q - Q_hi); this is exact for every element within a
+// factor 2^-9 of the row maximum (smaller ones carry an absolute error of at
+// most 2^-16 of the maximum).  B = [Q_hi ; Q_lo] is one N=128 operand, so S_hi and S_lo
+// come out of one MMA and the softmax adds them.  The softmax weights are
+// scaled by 2^7, p' = 2^(s - m + 7), and split the same way, P = P_hi + P_lo:
+// about 8 significant bits (like bf16) for every p' >= 2^-2 and an absolute
+// error of at most 2^-9 for smaller weights.  PV accumulates both terms; the scale
+// cancels in O / l and is removed from the LSE.
 //
-// Online softmax (log2 domain, scores pre-multiplied by log2 e): the running
-// max m per row only grows; when it grows, the O^T columns and the row sums
-// are rescaled by 2^(m_old - m_new) before the next PV accumulates.
+// Online softmax (log2 domain, scores pre-multiplied by log2 e), with a lazy
+// running max: the max m used for a row only moves when a tile's max exceeds
+// it by more than 1 (a factor of 2), so p' stays <= 2^8 and rescaling of the
+// O^T columns and row sums (by 2^(m_old - m_new)) is rare.
 //
 // Warp roles (512 threads):
-//   warp 0        TMA producer: pages -> 64-byte-swizzled chunks
-//   warp 1        UMMA issuer (one thread) and TMEM owner
+//   warp 0        TMA producer: pages -> 64-byte-swizzled chunks, plus L2
+//                 prefetch of tiles up to three ahead
+//   warp 1        UMMA issuer (warp-uniform polling of readiness, so a ready
+//                 PV is never held behind QK data still in flight; one
+//                 elected lane issues) and TMEM owner
 //   warps 4-7     softmax, query columns 0-31   (thread = token row of S^T)
 //   warps 8-11    softmax, query columns 32-63
 //   warps 12-15   O^T rescaling between tiles, epilogue (thread = latent dim)
@@ -63,7 +67,8 @@ constexpr int kTile = 128;          // tokens per tile (UMMA M)
 constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
 constexpr int kRingPairs = 8;       // two tiles of latent dims in flight
-constexpr float kPShift = 8.0f;     // log2 of the factor carried by the softmax weights
+constexpr float kPShift = 7.0f;     // log2 of the factor carried by the softmax weights
+constexpr float kLazy = 1.0f;       // the used max moves only when exceeded by more than this
 
 constexpr int kOffQ = 0;                                 // 9 chunks, rows hi 0-63 | lo 64-127
 constexpr int kOffRing = kOffQ + 9 * kChunk;             // 73728
@@ -94,9 +99,9 @@ struct Scratch {
   int abort;
   int pad[2];
   float warp_max[2][4][32];  // per softmax group, per warp, per column; reused for row sums
-  float m_run[64];           // running max per column (log2 units)
+  float m_run[64];           // max used per column (log2 units)
   float alpha[2][64];        // per tile parity: rescale factor per column
-  uint32_t changed[2][2];    // per tile parity, per column half: columns whose max grew
+  uint32_t changed[2][2];    // per tile parity, per column half: columns whose max moved
   float c_head[64];          // per column: softmax_scale * kv_scale * log2(e) * 2^-e
   float inv_l[64];           // per column: kv_scale / l  (0 when l == 0)
   uint8_t qcol[64];          // per column: its query position q
@@ -114,16 +119,26 @@ __device__ __forceinline__ void set_error(int32_t* err, int bit) {
   if (err != nullptr) atomicOr(err, bit);
 }
 
-// Convert 8 scaled fp32 query values into 8 hi and 8 lo E4M3 codes.
+// Descriptor for a start address `bytes` past the one `base` encodes (the
+// start field holds address >> 4 in its low 14 bits; addresses stay below
+// 256 KiB, so the add never carries out of the field).
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t bytes) {
+  return base + (uint64_t)(bytes >> 4);
+}
+
+// Split 8 fp32 values into two E4M3 terms each: hi = x rounded to 4
+// significant bits (round half away from zero on the bit pattern; an exact
+// E4M3 value for |x| in the normal range), lo = E4M3(x - hi).  Result bytes
+// are in element order.
 __device__ __forceinline__ void split8(const float* x, uint2& hi, uint2& lo) {
   uint32_t h[4], l[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const uint32_t hc = cvt_e4m3x2(x[2 * k], x[2 * k + 1]);
-    const float2 back = half2_bits_to_float2(cvt_e4m3x2_to_f16x2((uint16_t)hc));
-    const uint32_t lc = cvt_e4m3x2(x[2 * k] - back.x, x[2 * k + 1] - back.y);
-    h[k] = hc;
-    l[k] = lc;
+    const float a = x[2 * k], b = x[2 * k + 1];
+    const float ha = __uint_as_float((__float_as_uint(a) + 0x80000u) & 0xFFF00000u);
+    const float hb = __uint_as_float((__float_as_uint(b) + 0x80000u) & 0xFFF00000u);
+    h[k] = cvt_e4m3x2(ha, hb);
+    l[k] = cvt_e4m3x2(a - ha, b - hb);
   }
   hi.x = h[0] | (h[1] << 16);
   hi.y = h[2] | (h[3] << 16);
@@ -223,136 +238,182 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================ TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&kv_map);
-      const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
-      int last_nope_parity[kRingPairs];
-      bool armed[kRingPairs];
-      for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
-      int rope_armed_tiles = 0;
-      bool ok = true;
-      for (int i = 0; i < T && ok; ++i) {
-        const int tok0 = t0 + i * kTile;
-        const int pa = bt[p0 + 2 * i];
-        const bool want_b = tok0 + 64 < t1;
-        const int pb = want_b ? bt[p0 + 2 * i + 1] : 0;
-        bool la = (pa >= 0 && (int64_t)pa < args.num_pages);
-        bool lb = want_b && (pb >= 0 && (int64_t)pb < args.num_pages);
-        if (!la || (want_b && !lb)) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
-        const uint32_t bytes_chunk = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
-        for (int j = 0; j < 4; ++j) {
-          const int slot = (i & 1) * 4 + j;
-          if (i >= 2 && !(ok = mbar_wait(&bars[kBarNopeEmpty + slot], ((i - 2) >> 1) & 1, abort_flag)))
-            break;
-          uint64_t* full = &bars[kBarNopeFull + slot];
-          mbar_arrive_expect_tx(full, 2 * bytes_chunk);
-          armed[slot] = true;
-          last_nope_parity[slot] = (i >> 1) & 1;
-          uint8_t* dst = smem + kOffRing + slot * kPair;
-          for (int cc = 0; cc < 2; ++cc) {
-            const int chunk = 2 * j + cc;
-            if (la) tma_load_3d(dst + cc * kChunk, &kv_map, full, chunk * 64, 0, pa);
-            if (lb) tma_load_3d(dst + cc * kChunk + 4096, &kv_map, full, chunk * 64, 0, pb);
-          }
-        }
-        if (!ok) break;
-        if (i >= 1 && !(ok = mbar_wait(&bars[kBarRopeEmpty], (i - 1) & 1, abort_flag))) break;
-        uint64_t* rfull = &bars[kBarRopeFull];
-        mbar_arrive_expect_tx(rfull, bytes_chunk);
-        rope_armed_tiles = i + 1;
-        if (la) tma_load_3d(smem + kOffRope, &kv_map, rfull, 512, 0, pa);
-        if (lb) tma_load_3d(smem + kOffRope + 4096, &kv_map, rfull, 512, 0, pb);
+    // The whole warp runs this loop with warp-uniform values; one elected
+    // lane issues each TMA instruction and barrier arrival.
+    if (lane == 0) prefetch_tensormap(&kv_map);
+    __syncwarp();
+    const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
+    // L2 prefetch of a whole tile (both pages, all 9 chunks); page ids out of
+    // range are skipped here and reported by the load path
+    auto prefetch_tile = [&](int i) {
+      const int tok0 = t0 + i * kTile;
+      const int pa = bt[p0 + 2 * i];
+      const bool want_b = tok0 + 64 < t1;
+      const int pb = want_b ? bt[p0 + 2 * i + 1] : -1;
+      const bool ga = pa >= 0 && (int64_t)pa < args.num_pages;
+      const bool gb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
+      for (int c = 0; c < 9; ++c) {
+        if (ga) tma_prefetch_l2_3d_elect(&kv_map, c * 64, 0, pa);
+        if (gb) tma_prefetch_l2_3d_elect(&kv_map, c * 64, 0, pb);
       }
-      // drain: every armed transaction has landed before the CTA may exit
-      const uint64_t t_start = globaltimer_ns();
-      for (int i = 0; i < kRingPairs; ++i)
-        if (armed[i])
-          while (!mbar_try_wait(&bars[kBarNopeFull + i], last_nope_parity[i]) &&
-                 globaltimer_ns() - t_start < kWaitLimitNs) {
-          }
-      if (rope_armed_tiles > 0)
-        while (!mbar_try_wait(&bars[kBarRopeFull], (rope_armed_tiles - 1) & 1) &&
+    };
+    if (T > 2) prefetch_tile(2);
+    int last_nope_parity[kRingPairs];
+    bool armed[kRingPairs];
+    for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
+    int rope_armed_tiles = 0;
+    bool ok = true;
+    for (int i = 0; i < T && ok; ++i) {
+      if (i + 3 < T) prefetch_tile(i + 3);
+      const int tok0 = t0 + i * kTile;
+      const int pa = bt[p0 + 2 * i];
+      const bool want_b = tok0 + 64 < t1;
+      const int pb = want_b ? bt[p0 + 2 * i + 1] : 0;
+      const bool la = pa >= 0 && (int64_t)pa < args.num_pages;
+      const bool lb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
+      if (lane == 0 && (!la || (want_b && !lb))) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
+      const uint32_t bytes_chunk = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
+      for (int j = 0; j < 4; ++j) {
+        const int slot = (i & 1) * 4 + j;
+        if (i >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&bars[kBarNopeEmpty + slot], ((i - 2) >> 1) & 1, abort_flag));
+          if (!ok) break;
+        }
+        uint64_t* full = &bars[kBarNopeFull + slot];
+        mbar_arrive_expect_tx_elect(full, 2 * bytes_chunk);
+        armed[slot] = true;
+        last_nope_parity[slot] = (i >> 1) & 1;
+        uint8_t* dst = smem + kOffRing + slot * kPair;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int chunk = 2 * j + cc;
+          if (la) tma_load_3d_elect(dst + cc * kChunk, &kv_map, full, chunk * 64, 0, pa);
+          if (lb) tma_load_3d_elect(dst + cc * kChunk + 4096, &kv_map, full, chunk * 64, 0, pb);
+        }
+      }
+      if (!ok) break;
+      if (i >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarRopeEmpty], (i - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      uint64_t* rfull = &bars[kBarRopeFull];
+      mbar_arrive_expect_tx_elect(rfull, bytes_chunk);
+      rope_armed_tiles = i + 1;
+      if (la) tma_load_3d_elect(smem + kOffRope, &kv_map, rfull, 512, 0, pa);
+      if (lb) tma_load_3d_elect(smem + kOffRope + 4096, &kv_map, rfull, 512, 0, pb);
+    }
+    // drain: every armed transaction has landed before the CTA may exit
+    const uint64_t t_start = globaltimer_ns();
+    for (int i = 0; i < kRingPairs; ++i)
+      if (armed[i])
+        while (!mbar_try_wait(&bars[kBarNopeFull + i], last_nope_parity[i]) &&
                globaltimer_ns() - t_start < kWaitLimitNs) {
         }
-    }
+    if (rope_armed_tiles > 0)
+      while (!mbar_try_wait(&bars[kBarRopeFull], (rope_armed_tiles - 1) & 1) &&
+             globaltimer_ns() - t_start < kWaitLimitNs) {
+      }
   } else if (warp == 1) {
     // ============================================================ UMMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, 128, 128);  // E4M3 K-major x K-major, N=128
-      const uint32_t idesc_pv = instr_desc(0, 0, 1, 1, 128, 64);   // MN-major x MN-major, N=64
-      const uint32_t sQ = smem_u32(smem + kOffQ);
-      const uint32_t sRing = smem_u32(smem + kOffRing);
-      const uint32_t sRope = smem_u32(smem + kOffRope);
-      const uint32_t sPhi = smem_u32(smem + kOffPhi);
-      const uint32_t sPlo = smem_u32(smem + kOffPlo);
-      bool ok = mbar_wait(&bars[kBarQReady], 0, abort_flag);
-      tc_fence_after();
-      for (int i = 0; i <= T && ok; ++i) {
-        if (i < T) {
-          // ---------------- S^T(i) = K(i) . [Q_hi ; Q_lo]^T
-          const int sb = i & 1;
-          const uint32_t d_s = tmem + sb * 128;
-          if (i >= 2 && !(ok = mbar_wait(&bars[kBarSEmpty + sb], ((i - 2) >> 1) & 1, abort_flag)))
-            break;
+    // Warp-uniform scheduler; one elected lane issues each MMA and commit.
+    const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, 128, 128);  // E4M3 K-major x K-major, N=128
+    const uint32_t idesc_pv = instr_desc(0, 0, 1, 1, 128, 64);   // MN-major x MN-major, N=64
+    // K-major SW64 (8-row groups 512 B apart) and MN-major SW64 (64-element
+    // atoms 8 KiB apart, 8-row groups 512 B apart) descriptor bases
+    const uint64_t dRingK = smem_desc(smem_u32(smem + kOffRing), 16, 512, 4);
+    const uint64_t dRope = smem_desc(smem_u32(smem + kOffRope), 16, 512, 4);
+    const uint64_t dQ = smem_desc(smem_u32(smem + kOffQ), 16, 512, 4);
+    const uint64_t dRingMN = smem_desc(smem_u32(smem + kOffRing), kChunk, 512, 4);
+    const uint64_t dPhi = smem_desc(smem_u32(smem + kOffPhi), kChunk, 512, 4);
+    const uint64_t dPlo = smem_desc(smem_u32(smem + kOffPlo), kChunk, 512, 4);
+    auto ready = [&](int bar, int parity) {
+      return __any_sync(0xffffffffu, mbar_test_wait(&bars[bar], parity));
+    };
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQReady], 0, abort_flag));
+    tc_fence_after();
+    int nq = 0, qpair = 0, np = 0;
+    bool s_free = false;
+    uint64_t idle_since = 0;
+    uint32_t idle_spins = 0;
+    while (ok && np < T) {
+      bool progress = false;
+      // ---------------- S^T(nq) = K(nq) . [Q_hi ; Q_lo]^T, one 128-dim pair at a time
+      if (nq < T) {
+        const int sb = nq & 1;
+        const uint32_t d_s = tmem + sb * 128;
+        if (!s_free) {
+          s_free = nq < 2 || ready(kBarSEmpty + sb, ((nq - 2) >> 1) & 1);
+          if (s_free) tc_fence_after();
+        }
+        while (s_free && qpair < 4 && ready(kBarNopeFull + (nq & 1) * 4 + qpair, (nq >> 1) & 1)) {
           tc_fence_after();
-          for (int j = 0; j < 4 && ok; ++j) {
-            const int slot = (i & 1) * 4 + j;
-            if (!(ok = mbar_wait(&bars[kBarNopeFull + slot], (i >> 1) & 1, abort_flag))) break;
-            tc_fence_after();
+          const uint32_t a_off = ((nq & 1) * 4 + qpair) * kPair;
+          const uint32_t b_off = 2 * qpair * kChunk;
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const uint32_t a_base = sRing + slot * kPair + cc * kChunk;
-              const uint32_t b_base = sQ + (2 * j + cc) * kChunk;
+          for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-              for (int kk = 0; kk < 2; ++kk)
-                umma_f8(d_s, smem_desc(a_base + kk * 32, 16, 512, 4),
-                        smem_desc(b_base + kk * 32, 16, 512, 4), idesc_qk,
-                        (j | cc | kk) != 0 ? 1u : 0u);
-            }
-          }
-          if (!ok) break;
-          if (!(ok = mbar_wait(&bars[kBarRopeFull], i & 1, abort_flag))) break;
+            for (int kk = 0; kk < 2; ++kk)
+              umma_f8_elect(d_s, desc_at(dRingK, a_off + cc * kChunk + kk * 32),
+                            desc_at(dQ, b_off + cc * kChunk + kk * 32), idesc_qk,
+                            (qpair | cc | kk) != 0 ? 1u : 0u);
+          ++qpair;
+          progress = true;
+        }
+        if (s_free && qpair == 4 && ready(kBarRopeFull, nq & 1)) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            umma_f8(d_s, smem_desc(sRope + kk * 32, 16, 512, 4),
-                    smem_desc(sQ + 8 * kChunk + kk * 32, 16, 512, 4), idesc_qk, 1u);
-          umma_commit(&bars[kBarSFull + sb]);
-          umma_commit(&bars[kBarRopeEmpty]);
+            umma_f8_elect(d_s, desc_at(dRope, kk * 32), desc_at(dQ, 8 * kChunk + kk * 32),
+                          idesc_qk, 1u);
+          umma_commit_elect(&bars[kBarSFull + sb]);
+          umma_commit_elect(&bars[kBarRopeEmpty]);
+          ++nq;
+          qpair = 0;
+          s_free = false;
+          progress = true;
         }
-        if (i >= 1) {
-          // ---------------- O^T += V(k)^T . (P_hi + P_lo)
-          const int k = i - 1;
-          if (!(ok = mbar_wait(&bars[kBarPFull], k & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(&bars[kBarOReady], k & 1, abort_flag))) break;
-          tc_fence_after();
-          // the four O^T blocks are independent accumulators: issue them round-robin
-          // so that consecutive MMAs never wait on each other's accumulation
+      }
+      // ---------------- O^T += V(np)^T . (P_hi + P_lo)
+      if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady, np & 1)) {
+        tc_fence_after();
+        const uint32_t slot0 = (np & 1) * 4 * kPair;
+        // the four O^T blocks are independent accumulators, issued round-robin
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-            for (int hl = 0; hl < 2; ++hl) {
-              const uint64_t bdesc = smem_desc((hl ? sPlo : sPhi) + kk * 2048, kChunk, 512, 4);
+          for (int hl = 0; hl < 2; ++hl) {
+            const uint64_t bdesc = desc_at(hl ? dPlo : dPhi, kk * 2048);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int slot = (k & 1) * 4 + j;
-                const uint64_t a = smem_desc(sRing + slot * kPair + kk * 2048, kChunk, 512, 4);
-                umma_f8(tmem + 256 + 64 * j, a, bdesc, idesc_pv,
-                        (k > 0 || kk > 0 || hl > 0) ? 1u : 0u);
-              }
-            }
+            for (int j = 0; j < 4; ++j)
+              umma_f8_elect(tmem + 256 + 64 * j, desc_at(dRingMN, slot0 + j * kPair + kk * 2048),
+                            bdesc, idesc_pv, (np > 0 || kk > 0 || hl > 0) ? 1u : 0u);
           }
-          umma_commit(&bars[kBarPEmpty]);
+        }
+        umma_commit_elect(&bars[kBarPEmpty]);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) umma_commit(&bars[kBarNopeEmpty + (k & 1) * 4 + j]);
-          umma_commit(&bars[kBarPvDone]);
+        for (int j = 0; j < 4; ++j) umma_commit_elect(&bars[kBarNopeEmpty + (np & 1) * 4 + j]);
+        umma_commit_elect(&bars[kBarPvDone]);
+        ++np;
+        progress = true;
+      }
+      if (progress) {
+        idle_spins = 0;
+      } else if ((++idle_spins & 63) == 0) {
+        const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
+        if (idle_spins == 64) idle_since = now;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+          ok = false;
+        } else if (now - idle_since > kWaitLimitNs) {
+          if (lane == 0) *abort_flag = 1;
+          ok = false;
         }
       }
-      // drain: all issued MMAs complete before TMEM is released
-      umma_commit(&bars[kBarDrain]);
-      const uint64_t t_start = globaltimer_ns();
-      while (!mbar_try_wait(&bars[kBarDrain], 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
-      }
+    }
+    // drain: all issued MMAs complete before TMEM is released
+    umma_commit_elect(&bars[kBarDrain]);
+    const uint64_t t_start = globaltimer_ns();
+    while (!mbar_try_wait(&bars[kBarDrain], 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
     }
   } else if (warp >= 4 && warp < 12) {
     // ============================================================ Q split + softmax
@@ -366,26 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint16_t* qn = args.q_nope + (row_base + n) * 512;
         const uint16_t* qr = args.q_rope + (row_base + n) * 64;
         uint4 v[3];
-        int nch = 0;
-        int dim0[3];
-        if (valid) {
-          v[0] = *reinterpret_cast<const uint4*>(qn + lane * 8);
-          dim0[0] = lane * 8;
-          v[1] = *reinterpret_cast<const uint4*>(qn + 256 + lane * 8);
-          dim0[1] = 256 + lane * 8;
-          nch = 2;
-          if (lane < 8) {
-            v[2] = *reinterpret_cast<const uint4*>(qr + lane * 8);
-            dim0[2] = 512 + lane * 8;
-            nch = 3;
-          }
-        } else {
-          v[0] = v[1] = v[2] = make_uint4(0, 0, 0, 0);
-          dim0[0] = lane * 8;
-          dim0[1] = 256 + lane * 8;
-          dim0[2] = 512 + lane * 8;
-          nch = lane < 8 ? 3 : 2;
-        }
+        const int nch = lane < 8 ? 3 : 2;
+        const int dim0[3] = {lane * 8, 256 + lane * 8, 512 + lane * 8};
+        v[0] = valid ? *reinterpret_cast<const uint4*>(qn + lane * 8) : make_uint4(0, 0, 0, 0);
+        v[1] = valid ? *reinterpret_cast<const uint4*>(qn + 256 + lane * 8) : make_uint4(0, 0, 0, 0);
+        v[2] = (valid && lane < 8) ? *reinterpret_cast<const uint4*>(qr + lane * 8)
+                                   : make_uint4(0, 0, 0, 0);
         uint32_t amax_bits = 0;
         for (int c = 0; c < nch; ++c) {
           const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
@@ -434,23 +481,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = wq * 32 + lane;
     const int col0 = wg * 32;
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-    float c_reg[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) c_reg[j] = sc.c_head[col0 + j];
+    const float4* c4 = reinterpret_cast<const float4*>(sc.c_head + col0);
     float l_part[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) l_part[j] = 0.0f;
     const int bar_id = 1 + wg;
     bool ok = true;
+    bool bad = false;
     for (int i = 0; i < T; ++i) {
       const int sb = i & 1;
       const int tok = t0 + i * kTile + r;
-      // one leader waits, the group follows after a named barrier (uniform outcome)
-      if (wq == 0 && lane == 0) mbar_wait(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag);
-      if (named_bar_or(bar_id, 128, *abort_flag != 0)) {
-        ok = false;
-        break;
-      }
+      bad |= !mbar_wait(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag);
       tc_fence_after();
       float sv[32];
       {
@@ -459,7 +500,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16x2(ts, ts + 16, hi, hi + 16);
         tmem_ld16x2(ts + 64, ts + 64 + 16, lo, lo + 16);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sv[j] = (hi[j] + lo[j]) * c_reg[j];
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 c = c4[j4];
+          sv[4 * j4 + 0] = (hi[4 * j4 + 0] + lo[4 * j4 + 0]) * c.x;
+          sv[4 * j4 + 1] = (hi[4 * j4 + 1] + lo[4 * j4 + 1]) * c.y;
+          sv[4 * j4 + 2] = (hi[4 * j4 + 2] + lo[4 * j4 + 2]) * c.z;
+          sv[4 * j4 + 3] = (hi[4 * j4 + 3] + lo[4 * j4 + 3]) * c.w;
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars[kBarSEmpty + sb]);
@@ -478,59 +525,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         mine = (lane == j) ? wm : mine;
       }
       sc.warp_max[wg][wq][lane] = mine;
-      named_bar_sync(bar_id, 128);
+      if (named_bar_or(bar_id, 128, bad || *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
       if (wq == 0) {
         const int n = col0 + lane;
         const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
                                fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
         const float m_old = sc.m_run[n];
-        const float m_new = fmaxf(m_old, tm);
-        const bool grew = m_new > m_old;
-        const float a = grew ? (m_old == -INFINITY ? 0.0f : exp2f(m_old - m_new)) : 1.0f;
+        const bool moved = tm > m_old + kLazy;
+        const float m_new = moved ? tm : m_old;
+        const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
         sc.m_run[n] = m_new;
         sc.alpha[i & 1][n] = a;
-        const uint32_t mask = __ballot_sync(0xffffffffu, grew);
+        const uint32_t mask = __ballot_sync(0xffffffffu, moved);
         if (lane == 0) sc.changed[i & 1][wg] = mask;
       }
       named_bar_sync(bar_id, 128);
       if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull]);
-      // P buffer free (PV of the previous tile done)
-      if (i >= 1) {
-        if (wq == 0 && lane == 0) mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
-        if (named_bar_or(bar_id, 128, *abort_flag != 0)) {
-          ok = false;
-          break;
-        }
-      }
-      uint32_t phi[8], plo[8];
+      const float4* m4 = reinterpret_cast<const float4*>(sc.m_run + col0);
+      const float4* a4 = reinterpret_cast<const float4*>(sc.alpha[i & 1] + col0);
+      uint2 phi[4], plo[4];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float m0 = sc.m_run[col0 + j], m1 = sc.m_run[col0 + j + 1];
-        const float a0 = sc.alpha[i & 1][col0 + j], a1 = sc.alpha[i & 1][col0 + j + 1];
-        // weights carry a 2^8 factor: p' = 2^(s - m + 8) in (0, 256], so that both
-        // E4M3 terms of every p' >= 2^-2 are normal numbers
-        const float p0v = (sv[j] == -INFINITY) ? 0.0f : exp2f(sv[j] - m0 + kPShift);
-        const float p1v = (sv[j + 1] == -INFINITY) ? 0.0f : exp2f(sv[j + 1] - m1 + kPShift);
-        l_part[j] = fmaf(l_part[j], a0, p0v);
-        l_part[j + 1] = fmaf(l_part[j + 1], a1, p1v);
-        const uint32_t hc = cvt_e4m3x2(p0v, p1v);
-        const float2 back = half2_bits_to_float2(cvt_e4m3x2_to_f16x2((uint16_t)hc));
-        const uint32_t lc = cvt_e4m3x2(p0v - back.x, p1v - back.y);
-        if ((j & 2) == 0) {
-          phi[j >> 2] = hc;
-          plo[j >> 2] = lc;
-        } else {
-          phi[j >> 2] |= hc << 16;
-          plo[j >> 2] |= lc << 16;
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const float4 ma = m4[2 * q8], mb = m4[2 * q8 + 1];
+        const float4 aa = a4[2 * q8], ab = a4[2 * q8 + 1];
+        const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+        const float al[8] = {aa.x, aa.y, aa.z, aa.w, ab.x, ab.y, ab.z, ab.w};
+        float pv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int j = 8 * q8 + k;
+          // weights carry a 2^7 factor: p' = 2^(s - m + 7) <= 2^8
+          pv[k] = (sv[j] == -INFINITY) ? 0.0f : ex2_approx(sv[j] - mm[k] + kPShift);
+          l_part[j] = fmaf(l_part[j], al[k], pv[k]);
         }
+        split8(pv, phi[q8], plo[q8]);
       }
+      // P buffer (and the V rows cleared below) free: PV of the previous tile done
+      if (i >= 1) bad |= !mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
       {
         uint8_t* ph = smem + kOffPhi;
         uint8_t* pl = smem + kOffPlo;
-        *reinterpret_cast<uint4*>(ph + sw64(r, col0)) = make_uint4(phi[0], phi[1], phi[2], phi[3]);
-        *reinterpret_cast<uint4*>(ph + sw64(r, col0 + 16)) = make_uint4(phi[4], phi[5], phi[6], phi[7]);
-        *reinterpret_cast<uint4*>(pl + sw64(r, col0)) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
-        *reinterpret_cast<uint4*>(pl + sw64(r, col0 + 16)) = make_uint4(plo[4], plo[5], plo[6], plo[7]);
+        *reinterpret_cast<uint4*>(ph + sw64(r, col0)) = make_uint4(phi[0].x, phi[0].y, phi[1].x, phi[1].y);
+        *reinterpret_cast<uint4*>(ph + sw64(r, col0 + 16)) = make_uint4(phi[2].x, phi[2].y, phi[3].x, phi[3].y);
+        *reinterpret_cast<uint4*>(pl + sw64(r, col0)) = make_uint4(plo[0].x, plo[0].y, plo[1].x, plo[1].y);
+        *reinterpret_cast<uint4*>(pl + sw64(r, col0 + 16)) = make_uint4(plo[2].x, plo[2].y, plo[3].x, plo[3].y);
       }
       if (tok >= t1) {
         // rows past the visible range: clear their V bytes so 0 * garbage cannot be NaN
