@@ -80,7 +80,39 @@ def test_decode_reports_bad_page_ids():
     assert err & m.DEVERR_BAD_PAGE
 
 
-FULL = [("b1_128k_fp8", 64), ("b16_128k_fp8", 32), ("verify_q4_256k_fp8", 24)]
+BF16 = [
+    ("tiny", {}),                                                   # the tiny workload as specified
+    ("tiny", dict(seq_lens=[1], splits=1)),
+    ("tiny", dict(seq_lens=[129], splits=2)),
+    ("tiny", dict(seq_lens=[100], splits=8)),                       # more splits than pages
+    ("tiny", dict(seq_lens=[777, 64, 2000], splits=3, H=64)),
+    ("tiny", dict(seq_lens=[1000], splits=2, H=64, q_len=4)),       # causal, four row groups
+    ("tiny", dict(seq_lens=[555], splits=3, H=16, q_len=4)),        # causal inside one group
+    ("b32_ragged_bf16", dict(seq_lens=[300, 4100, 70], splits=2)),  # 128 heads: two row groups
+]
+
+
+@pytest.mark.parametrize("case", BF16, ids=[_ids(c) for c in BF16])
+def test_decode_bf16_small_matches_oracle(case):
+    spec, ov = case
+    c = make_case(spec, **ov)
+    w = c.w
+    out, lse, part_o, part_lse, err = run_gpu(c)
+    assert err == 0
+    rows = np.arange(w.B * w.q_len * w.H)
+    o_ref, l_ref = oracle_rows(c, rows)
+    assert_attention_close(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
+                           o_ref, l_ref, what=str(case))
+    po_ref, pl_ref = oracle_partials(c, rows)
+    pl = part_lse.cpu().numpy().reshape(len(rows), w.max_splits)
+    ns = w.num_splits.cpu().numpy()[rows // (w.q_len * w.H)]
+    for r in range(len(rows)):
+        S = ns[r]
+        assert np.array_equal(np.isneginf(pl[r, :S]), np.isneginf(pl_ref[r, :S])), r
+
+
+FULL = [("b1_128k_fp8", 64), ("b16_128k_fp8", 32), ("verify_q4_256k_fp8", 24),
+        ("b32_ragged_bf16", 32)]
 
 
 @pytest.mark.parametrize("spec,n_rows", FULL)
