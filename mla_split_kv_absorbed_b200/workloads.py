@@ -74,6 +74,8 @@ SPECS = {
     # profiling size: the batch-16 shape cut to 4 requests (302 MB of KV, > L2)
     "b4_128k_fp8": Spec("b4_128k_fp8", B=4, q_len=1, H=64, seq_lens=[131072] * 4,
                         kv_dtype="fp8", kv_std=1.0, splits=32, seed=5),
+    "b4_128k_bf16": Spec("b4_128k_bf16", B=4, q_len=1, H=64, seq_lens=[131072] * 4,
+                         kv_dtype="bf16", kv_std=1.0, splits=32, seed=5),
     "verify_q4_256k_fp8": Spec("verify_q4_256k_fp8", B=8, q_len=4, H=64,
                                seq_lens=[262144] * 8, kv_dtype="fp8", kv_std=1.0, splits=64,
                                seed=4),
