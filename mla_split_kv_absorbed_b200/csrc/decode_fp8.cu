@@ -39,16 +39,18 @@
 // it by more than 1 (a factor of 2), so p' stays <= 2^8 and rescaling of the
 // O^T columns and row sums (by 2^(m_old - m_new)) is rare.
 //
-// Warp roles (512 threads):
+// Warp roles (768 threads):
 //   warp 0        TMA producer: pages -> 64-byte-swizzled chunks, plus L2
 //                 prefetch of tiles up to three ahead
 //   warp 1        UMMA issuer (warp-uniform polling of readiness, so a ready
 //                 PV is never held behind QK data still in flight; one
 //                 elected lane issues) and TMEM owner
-//   warps 4-7     softmax, query columns 0-31   (thread = token row of S^T)
-//   warps 8-11    softmax, query columns 32-63
-//   warps 12-15   O^T rescaling between tiles, epilogue (thread = latent dim)
-//   warps 4-11    also convert Q to the split FP8 operand at the start
+//   warps 4-19    softmax in four warpgroups of 16 query columns each
+//                 (thread = token row of S^T); the softmax of a tile is on
+//                 the critical path of the two-tile ring, so it gets the
+//                 most warps that the register file allows
+//   warps 20-23   O^T rescaling between tiles, epilogue (thread = latent dim)
+//   warps 4-19    also convert Q to the split FP8 operand at the start
 // TMEM (512 columns): S^T buffers at 0 and 128 (S_hi 0-63 | S_lo 64-127),
 // O^T blocks at 256 + 64*j.
 #include <cstdint>
@@ -61,7 +63,10 @@
 namespace mla {
 namespace fp8k {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 768;
+constexpr int kSoftGroups = 4;      // softmax warpgroups
+constexpr int kCols = 16;           // query columns per softmax warpgroup
+constexpr int kSoftThreads = 128 * kSoftGroups;
 constexpr int kRows = 64;           // query rows per CTA (UMMA N for PV)
 constexpr int kTile = 128;          // tokens per tile (UMMA M)
 constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
@@ -98,10 +103,10 @@ struct Scratch {
   uint32_t tmem_base;
   int abort;
   int pad[2];
-  float warp_max[2][4][32];  // per softmax group, per warp, per column; reused for row sums
+  float warp_max[4][4][16];  // per softmax group, per warp, per column; reused for row sums
   float m_run[64];           // max used per column (log2 units)
   float alpha[2][64];        // per tile parity: rescale factor per column
-  uint32_t changed[2][2];    // per tile parity, per column half: columns whose max moved
+  uint32_t changed[2][4];    // per tile parity, per softmax group: columns whose max moved
   float c_head[64];          // per column: softmax_scale * kv_scale * log2(e) * 2^-e
   float inv_l[64];           // per column: kv_scale / l  (0 when l == 0)
   uint8_t qcol[64];          // per column: its query position q
@@ -209,14 +214,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sc.bars[kBarRopeEmpty], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sc.bars[kBarSFull + i], 1);
-      mbar_init(&sc.bars[kBarSEmpty + i], 256);
+      mbar_init(&sc.bars[kBarSEmpty + i], kSoftThreads);
     }
-    mbar_init(&sc.bars[kBarPFull], 256);
+    mbar_init(&sc.bars[kBarPFull], kSoftThreads);
     mbar_init(&sc.bars[kBarPEmpty], 1);
     mbar_init(&sc.bars[kBarOReady], 128);
     mbar_init(&sc.bars[kBarPvDone], 1);
-    mbar_init(&sc.bars[kBarQReady], 8);
-    mbar_init(&sc.bars[kBarAlphaFull], 2);
+    mbar_init(&sc.bars[kBarQReady], 4 * kSoftGroups);
+    mbar_init(&sc.bars[kBarAlphaFull], kSoftGroups);
     mbar_init(&sc.bars[kBarDrain], 1);
     sc.abort = 0;
     fence_barrier_init();
@@ -378,21 +383,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady, np & 1)) {
         tc_fence_after();
         const uint32_t slot0 = (np & 1) * 4 * kPair;
-        // the four O^T blocks are independent accumulators, issued round-robin
+        // block by block, so each latent pair can be refilled as soon as its
+        // block is done
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int j = 0; j < 4; ++j) {
 #pragma unroll
-          for (int hl = 0; hl < 2; ++hl) {
-            const uint64_t bdesc = desc_at(hl ? dPlo : dPhi, kk * 2048);
+          for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int hl = 0; hl < 2; ++hl)
               umma_f8_elect(tmem + 256 + 64 * j, desc_at(dRingMN, slot0 + j * kPair + kk * 2048),
-                            bdesc, idesc_pv, (np > 0 || kk > 0 || hl > 0) ? 1u : 0u);
-          }
+                            desc_at(hl ? dPlo : dPhi, kk * 2048), idesc_pv,
+                            (np > 0 || kk > 0 || hl > 0) ? 1u : 0u);
+          // latent pair j of this tile is free once its block's MMAs complete
+          umma_commit_elect(&bars[kBarNopeEmpty + (np & 1) * 4 + j]);
         }
         umma_commit_elect(&bars[kBarPEmpty]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) umma_commit_elect(&bars[kBarNopeEmpty + (np & 1) * 4 + j]);
         umma_commit_elect(&bars[kBarPvDone]);
         ++np;
         progress = true;
@@ -415,14 +420,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t t_start = globaltimer_ns();
     while (!mbar_try_wait(&bars[kBarDrain], 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < 4 + 4 * kSoftGroups) {
     // ============================================================ Q split + softmax
-    const int wg = (warp - 4) >> 2;  // 0: columns 0-31, 1: columns 32-63
+    const int wg = (warp - 4) >> 2;  // softmax group: query columns 16*wg .. 16*wg+15
     const int wq = warp & 3;         // TMEM lane quadrant
     {
       // ---- Q -> [Q_hi ; Q_lo] in K-major SW64 chunks, per-row power-of-two scale
-      const int pw = warp - 4;  // 0..7, rows pw, pw+8, ...
-      for (int n = pw; n < kRows; n += 8) {
+      const int pw = warp - 4;  // rows pw, pw + 16, ...
+      for (int n = pw; n < kRows; n += 4 * kSoftGroups) {
         const bool valid = n < rows_valid;
         const uint16_t* qn = args.q_nope + (row_base + n) * 512;
         const uint16_t* qr = args.q_rope + (row_base + n) * 64;
@@ -447,8 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int e = 0;
         if (amax > 0.0f && amax_bits < 0x7F800000u) {
           int E;
-          frexpf(amax, &E);
-          e = min(max(8 - E, -126), 126);
+          frexpf(amax, &E);    // amax in [2^(E-1), 2^E)
+          e = min(max(8 - E, -126), 126);  // amax * 2^e in [128, 256)
         }
         const float sc_up = __uint_as_float((uint32_t)(127 + e) << 23);
         for (int c = 0; c < nch; ++c) {
@@ -474,17 +479,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarQReady]);
-      named_bar_sync(5, 256);  // c_head visible to both softmax groups
+      named_bar_sync(7, kSoftThreads);  // c_head visible to every softmax group
     }
 
-    // ---- softmax over S^T: thread = token row r of the tile
+    // ---- softmax over S^T: thread = token row r of the tile, 16 query columns
     const int r = wq * 32 + lane;
-    const int col0 = wg * 32;
+    const int col0 = wg * kCols;
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     const float4* c4 = reinterpret_cast<const float4*>(sc.c_head + col0);
-    float l_part[32];
+    float l_part[kCols];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) l_part[j] = 0.0f;
+    for (int j = 0; j < kCols; ++j) l_part[j] = 0.0f;
     const int bar_id = 1 + wg;
     bool ok = true;
     bool bad = false;
@@ -493,14 +498,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tok = t0 + i * kTile + r;
       bad |= !mbar_wait(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag);
       tc_fence_after();
-      float sv[32];
+      float sv[kCols];
       {
-        float hi[32], lo[32];
+        float hi[kCols], lo[kCols];
         const uint32_t ts = t_lane + sb * 128 + col0;
-        tmem_ld16x2(ts, ts + 16, hi, hi + 16);
-        tmem_ld16x2(ts + 64, ts + 64 + 16, lo, lo + 16);
+        tmem_ld16x2(ts, ts + 64, hi, lo);
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
+        for (int j4 = 0; j4 < kCols / 4; ++j4) {
           const float4 c = c4[j4];
           sv[4 * j4 + 0] = (hi[4 * j4 + 0] + lo[4 * j4 + 0]) * c.x;
           sv[4 * j4 + 1] = (hi[4 * j4 + 1] + lo[4 * j4 + 1]) * c.y;
@@ -514,31 +518,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t0 + i * kTile + kTile > t_all) {
         const int qq = tok - vis_base;  // token invisible to columns whose q <= qq
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < kCols; ++j)
           if (tok >= t1 || (qq >= 0 && (int)sc.qcol[col0 + j] <= qq)) sv[j] = -INFINITY;
       }
       // per-column tile max: warp redux, then across the 4 warps
       float mine = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < kCols; ++j) {
         const float wm = warp_max_f32(sv[j]);
         mine = (lane == j) ? wm : mine;
       }
-      sc.warp_max[wg][wq][lane] = mine;
+      if (lane < kCols) sc.warp_max[wg][wq][lane] = mine;
       if (named_bar_or(bar_id, 128, bad || *abort_flag != 0)) {
         ok = false;
         break;
       }
       if (wq == 0) {
         const int n = col0 + lane;
-        const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
-                               fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
-        const float m_old = sc.m_run[n];
-        const bool moved = tm > m_old + kLazy;
-        const float m_new = moved ? tm : m_old;
-        const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
-        sc.m_run[n] = m_new;
-        sc.alpha[i & 1][n] = a;
+        bool moved = false;
+        if (lane < kCols) {
+          const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
+                                 fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
+          const float m_old = sc.m_run[n];
+          moved = tm > m_old + kLazy;
+          const float m_new = moved ? tm : m_old;
+          const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
+          sc.m_run[n] = m_new;
+          sc.alpha[i & 1][n] = a;
+        }
         const uint32_t mask = __ballot_sync(0xffffffffu, moved);
         if (lane == 0) sc.changed[i & 1][wg] = mask;
       }
@@ -546,9 +553,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull]);
       const float4* m4 = reinterpret_cast<const float4*>(sc.m_run + col0);
       const float4* a4 = reinterpret_cast<const float4*>(sc.alpha[i & 1] + col0);
-      uint2 phi[4], plo[4];
+      uint2 phi[kCols / 8], plo[kCols / 8];
 #pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
+      for (int q8 = 0; q8 < kCols / 8; ++q8) {
         const float4 ma = m4[2 * q8], mb = m4[2 * q8 + 1];
         const float4 aa = a4[2 * q8], ab = a4[2 * q8 + 1];
         const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
@@ -565,25 +572,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // P buffer (and the V rows cleared below) free: PV of the previous tile done
       if (i >= 1) bad |= !mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
-      {
-        uint8_t* ph = smem + kOffPhi;
-        uint8_t* pl = smem + kOffPlo;
-        *reinterpret_cast<uint4*>(ph + sw64(r, col0)) = make_uint4(phi[0].x, phi[0].y, phi[1].x, phi[1].y);
-        *reinterpret_cast<uint4*>(ph + sw64(r, col0 + 16)) = make_uint4(phi[2].x, phi[2].y, phi[3].x, phi[3].y);
-        *reinterpret_cast<uint4*>(pl + sw64(r, col0)) = make_uint4(plo[0].x, plo[0].y, plo[1].x, plo[1].y);
-        *reinterpret_cast<uint4*>(pl + sw64(r, col0 + 16)) = make_uint4(plo[2].x, plo[2].y, plo[3].x, plo[3].y);
-      }
+      *reinterpret_cast<uint4*>(smem + kOffPhi + sw64(r, col0)) =
+          make_uint4(phi[0].x, phi[0].y, phi[1].x, phi[1].y);
+      *reinterpret_cast<uint4*>(smem + kOffPlo + sw64(r, col0)) =
+          make_uint4(plo[0].x, plo[0].y, plo[1].x, plo[1].y);
       if (tok >= t1) {
         // rows past the visible range: clear their V bytes so 0 * garbage cannot be NaN
-        const int slot0 = (i & 1) * 4 + wg * 2;  // group 0 clears pairs 0-1, group 1 pairs 2-3
+        // (softmax group g clears latent pair g)
+        const int pair = (i & 1) * 4 + wg;
 #pragma unroll
-        for (int pp = 0; pp < 2; ++pp)
+        for (int cc = 0; cc < 2; ++cc) {
+          uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + pair * kPair + cc * kChunk + r * 64);
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + (slot0 + pp) * kPair + cc * kChunk + r * 64);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) row[u] = make_uint4(0, 0, 0, 0);
-          }
+          for (int u = 0; u < 4; ++u) row[u] = make_uint4(0, 0, 0, 0);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[kBarPFull]);
@@ -592,16 +594,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       float mine = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < kCols; ++j) {
         float v = l_part[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         mine = (lane == j) ? v : mine;
       }
       named_bar_sync(bar_id, 128);  // warp_max no longer read
-      sc.warp_max[wg][wq][lane] = mine;
+      if (lane < kCols) sc.warp_max[wg][wq][lane] = mine;
       named_bar_sync(bar_id, 128);
-      if (wq == 0) {
+      if (wq == 0 && lane < kCols) {
         const int n = col0 + lane;
         const float l = (sc.warp_max[wg][0][lane] + sc.warp_max[wg][1][lane]) +
                         (sc.warp_max[wg][2][lane] + sc.warp_max[wg][3][lane]);
@@ -612,29 +614,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               nonempty ? (sc.m_run[n] - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
     }
-    named_bar_sync(4, 384);  // inv_l ready for the epilogue
-  } else if (warp >= 12) {
+    named_bar_sync(6, kSoftThreads + 128);  // inv_l ready for the epilogue
+  } else if (warp >= 4 + 4 * kSoftGroups) {
     // ============================================================ O^T rescale + epilogue
     const int wq = warp & 3;
     const int d_lane = wq * 32 + lane;  // latent dim within a 128-wide block
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     bool ok = true;
     for (int i = 0; i < T; ++i) {
-      if (warp == 12 && lane == 0) {
+      if (wq == 0 && lane == 0) {
         mbar_wait(&bars[kBarAlphaFull], i & 1, abort_flag);
         if (i >= 1) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
       }
-      if (named_bar_or(3, 128, *abort_flag != 0)) {
+      if (named_bar_or(5, 128, *abort_flag != 0)) {
         ok = false;
         break;
       }
       tc_fence_after();
       if (i >= 1) {
         const uint32_t ch0 = sc.changed[i & 1][0], ch1 = sc.changed[i & 1][1];
-        if ((ch0 | ch1) != 0) {
+        const uint32_t ch2 = sc.changed[i & 1][2], ch3 = sc.changed[i & 1][3];
+        if ((ch0 | ch1 | ch2 | ch3) != 0) {
 #pragma unroll 1
-          for (int grp = 0; grp < 4; ++grp) {
-            const uint32_t bits = ((grp < 2 ? ch0 : ch1) >> ((grp & 1) * 16)) & 0xFFFFu;
+          for (int grp = 0; grp < 4; ++grp) {  // grp = softmax group = 16 columns
+            const uint32_t bits = grp == 0 ? ch0 : grp == 1 ? ch1 : grp == 2 ? ch2 : ch3;
             if (bits == 0) continue;
             float a[16];
 #pragma unroll
@@ -655,9 +658,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[kBarOReady]);
     }
-    if (ok && warp == 12 && lane == 0) mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
-    const bool bad = named_bar_or(3, 128, !ok || *abort_flag != 0);
-    named_bar_sync(4, 384);
+    if (ok && wq == 0 && lane == 0) mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
+    const bool bad = named_bar_or(5, 128, !ok || *abort_flag != 0);
+    named_bar_sync(6, kSoftThreads + 128);
     if (!bad) {
       tc_fence_after();
       float* po = args.part_o + (row_base * args.max_splits + s) * 512;
