@@ -49,7 +49,8 @@
 //                 (thread = token row of S^T); the softmax of a tile is on
 //                 the critical path of the two-tile ring, so it gets the
 //                 most warps that the register file allows
-//   warps 20-23   O^T rescaling between tiles, epilogue (thread = latent dim)
+//   warps 20-23   O^T rescaling between tiles (thread = latent dim)
+//   warps 4-23    epilogue: O^T / l from TMEM to the partial output
 //   warps 4-19    also convert Q to the split FP8 operand at the start
 // TMEM (512 columns): S^T buffers at 0 and 128 (S_hi 0-63 | S_lo 64-127),
 // O^T blocks at 256 + 64*j.
@@ -71,6 +72,7 @@ constexpr int kRows = 64;           // query rows per CTA (UMMA N for PV)
 constexpr int kTile = 128;          // tokens per tile (UMMA M)
 constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
+constexpr uint32_t kPageBytes = 64 * 576;  // one page of the pool
 constexpr int kRingPairs = 8;       // two tiles of latent dims in flight
 constexpr float kPShift = 7.0f;     // log2 of the factor carried by the softmax weights
 constexpr float kLazy = 1.0f;       // the used max moves only when exceeded by more than this
@@ -248,19 +250,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) prefetch_tensormap(&kv_map);
     __syncwarp();
     const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
-    // L2 prefetch of a whole tile (both pages, all 9 chunks); page ids out of
-    // range are skipped here and reported by the load path
+    // L2 prefetch of a whole tile: each page is one contiguous 36 KiB block,
+    // so one untiled bulk prefetch per page; page ids out of range are
+    // skipped here and reported by the load path
     auto prefetch_tile = [&](int i) {
       const int tok0 = t0 + i * kTile;
       const int pa = bt[p0 + 2 * i];
       const bool want_b = tok0 + 64 < t1;
       const int pb = want_b ? bt[p0 + 2 * i + 1] : -1;
-      const bool ga = pa >= 0 && (int64_t)pa < args.num_pages;
-      const bool gb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
-      for (int c = 0; c < 9; ++c) {
-        if (ga) tma_prefetch_l2_3d_elect(&kv_map, c * 64, 0, pa);
-        if (gb) tma_prefetch_l2_3d_elect(&kv_map, c * 64, 0, pb);
-      }
+      if (pa >= 0 && (int64_t)pa < args.num_pages)
+        bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pa * kPageBytes, kPageBytes);
+      if (want_b && pb >= 0 && (int64_t)pb < args.num_pages)
+        bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pb * kPageBytes, kPageBytes);
     };
     if (T > 2) prefetch_tile(2);
     int last_nope_parity[kRingPairs];
@@ -614,11 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               nonempty ? (sc.m_run[n] - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
     }
-    named_bar_sync(6, kSoftThreads + 128);  // inv_l ready for the epilogue
+    named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
   } else if (warp >= 4 + 4 * kSoftGroups) {
-    // ============================================================ O^T rescale + epilogue
-    const int wq = warp & 3;
-    const int d_lane = wq * 32 + lane;  // latent dim within a 128-wide block
+    // ============================================================ O^T rescale between tiles
+    const int wq = warp & 3;            // thread = latent dim wq * 32 + lane of a block
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     bool ok = true;
     for (int i = 0; i < T; ++i) {
@@ -659,23 +659,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars[kBarOReady]);
     }
     if (ok && wq == 0 && lane == 0) mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
-    const bool bad = named_bar_or(5, 128, !ok || *abort_flag != 0);
-    named_bar_sync(6, kSoftThreads + 128);
-    if (!bad) {
-      tc_fence_after();
+    named_bar_sync(5, 128);
+    tc_fence_before();
+    named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
+  }
+  if (warp >= 4) {
+    // ============================================================ epilogue (warps 4-23)
+    // O^T / l -> part_o, the sixteen [128 dims x 16 columns] TMEM chunks
+    // spread over the five warpgroups (thread = latent dim of a block)
+    tc_fence_after();
+    if (*abort_flag == 0) {
+      const int ewg = (warp - 4) >> 2;  // 0..4
+      const int wq = warp & 3;
+      const int d_lane = wq * 32 + lane;
+      const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
       float* po = args.part_o + (row_base * args.max_splits + s) * 512;
       const int64_t row_stride = (int64_t)args.max_splits * 512;
 #pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll 1
-        for (int grp = 0; grp < 4; ++grp) {
-          float v[16];
-          tmem_ld16(t_lane + 256 + 64 * j + 16 * grp, v);
+      for (int c = ewg; c < 16; c += 5) {
+        const int j = c >> 2, grp = c & 3;
+        float v[16];
+        tmem_ld16(t_lane + 256 + 64 * j + 16 * grp, v);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int n = grp * 16 + c;
-            if (n < rows_valid) po[n * row_stride + 128 * j + d_lane] = v[c] * sc.inv_l[n];
-          }
+        for (int cc = 0; cc < 16; ++cc) {
+          const int n = grp * 16 + cc;
+          if (n < rows_valid) po[n * row_stride + 128 * j + d_lane] = v[cc] * sc.inv_l[n];
         }
       }
     }

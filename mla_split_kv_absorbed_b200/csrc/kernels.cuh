@@ -17,6 +17,7 @@ cudaError_t launch_combine(const float* part_o, const float* part_lse, const int
 struct DecodeArgs {
   const uint16_t* q_nope;
   const uint16_t* q_rope;
+  const uint8_t* kv_pages;   // the page pool, [num_pages][64][576] elements
   const int32_t* block_table;
   const int32_t* seq_lens;
   const int32_t* num_splits;

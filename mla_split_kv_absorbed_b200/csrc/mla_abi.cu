@@ -124,6 +124,7 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   mla::DecodeArgs a;
   a.q_nope = q_nope;
   a.q_rope = q_rope;
+  a.kv_pages = static_cast<const uint8_t*>(kv_pages);
   a.block_table = block_table;
   a.seq_lens = seq_lens;
   a.num_splits = num_splits;

@@ -113,6 +113,16 @@ __device__ __forceinline__ void tma_prefetch_l2_3d_elect(const CUtensorMap* map,
       "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// Untiled bulk L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned
+// global address; one elected lane of the (converged) warp issues it.
+__device__ __forceinline__ void bulk_prefetch_l2_elect(const void* gaddr, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.prefetch.L2.global [%0], %1;\n\t}" ::"l"(gaddr),
+      "r"(bytes)
+      : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint64_t* bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
