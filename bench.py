@@ -142,7 +142,11 @@ def time_quantize(w, kv, reps=5):
 def run_steps(w, kv, steps, warmup, flush_bytes=256 << 20):
     """Time `steps` decode steps (partial + combine) with an L2 flush before each.
 
-    Returns per-step total device times and per-step partial-kernel times (s)."""
+    Returns per-step total device times and per-step partial-kernel times (s).
+    The totals come from steps bracketed by two events only, so nothing sits
+    between the two kernels on the stream (the merge kernel is a programmatic
+    dependent launch of the partial kernel); the partial-kernel times come from
+    a second set of steps with an event between the two kernels."""
     import torch
     import mla_split_kv_absorbed_b200 as m
     stream = torch.cuda.current_stream()
@@ -152,31 +156,38 @@ def run_steps(w, kv, steps, warmup, flush_bytes=256 << 20):
     flush = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def step(e_start=None, e_mid=None, e_end=None):
+        if e_start is not None:
+            e_start.record(stream)
         m.mla_decode_partial(w.q_nope, w.q_rope, kv, w.kv_scale, w.block_table, w.seq_lens,
                              w.num_splits, w.max_splits, w.softmax_scale, part_o, part_lse, err,
                              stream)
-        if ev is not None:
-            ev[1].record(stream)
+        if e_mid is not None:
+            e_mid.record(stream)
         m.mla_combine(part_o, part_lse, w.num_splits, w.max_splits, out, out_lse, stream)
-        if ev is not None:
-            ev[2].record(stream)
+        if e_end is not None:
+            e_end.record(stream)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
 
     for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    tot_ev = [(ev(), ev()) for _ in range(steps)]
     for i in range(steps):
         flush.zero_()
-        step(evs[i])
+        step(tot_ev[i][0], None, tot_ev[i][1])
+    par_ev = [(ev(), ev()) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        step(par_ev[i][0], par_ev[i][1], None)
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item())}")
-    total = [e[0].elapsed_time(e[2]) * 1e-3 for e in evs]
-    partial = [e[0].elapsed_time(e[1]) * 1e-3 for e in evs]
+    total = [a.elapsed_time(b) * 1e-3 for a, b in tot_ev]
+    partial = [a.elapsed_time(b) * 1e-3 for a, b in par_ev]
     return total, partial
 
 

@@ -11,7 +11,8 @@
 // Per row: M = max_s LSE_s, w_s = e^{LSE_s - M}, O = sum w_s O_s / sum w_s,
 // LSE = M + ln sum w_s.  Grid: (rows, 512 / 128), 128 threads; the split
 // weights of the row are computed once per block into shared memory while the
-// partial loads are in flight.
+// partial loads are in flight.  Up to 256 splits (two per thread for the
+// weights).
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -26,43 +27,56 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_lse,
     const int32_t* __restrict__ num_splits, int max_splits, int rows_per_batch,
     uint16_t* __restrict__ out, float* __restrict__ out_lse) {
-  extern __shared__ float w_smem[];  // [max_splits] weights, then [1] inverse sum
+  extern __shared__ float w_smem[];  // [max_splits] split weights
+  __shared__ float red[2][kCombineThreads / 32];
   const int row = blockIdx.x;
   const int d = blockIdx.y * kCombineThreads + threadIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int b = row / rows_per_batch;
   int S = num_splits[b];
   S = S < 0 ? 0 : (S > max_splits ? max_splits : S);
   const float* po = part_o + (size_t)row * max_splits * 512 + d;
+  const float* pl = part_lse + (size_t)row * max_splits;
+
+  // launched as a programmatic dependent of the partial kernel: everything
+  // above overlapped its tail; the partials are read only after it completes
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // issue the first group of partial loads before anything else
   float v[kCombineGroup];
 #pragma unroll
   for (int j = 0; j < kCombineGroup; ++j) v[j] = (j < S) ? __ldg(po + (size_t)j * 512) : 0.0f;
 
-  // split weights (overlaps the loads above)
-  const float* pl = part_lse + (size_t)row * max_splits;
-  __shared__ float red[kCombineThreads / 32];
-  float m = -INFINITY;
-  for (int s = threadIdx.x; s < S; s += kCombineThreads) m = fmaxf(m, pl[s]);
+  // split weights while those loads are in flight: M = max LSE, w_s = e^(LSE_s - M)
+  float lse[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int sidx = threadIdx.x + k * kCombineThreads;
+    lse[k] = sidx < S ? pl[sidx] : -INFINITY;
+  }
+  float m = fmaxf(lse[0], lse[1]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  if (lane == 0) red[0][wid] = m;
   __syncthreads();
-  m = red[0];
+  m = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+  float wpart = 0.0f;
 #pragma unroll
-  for (int i = 1; i < kCombineThreads / 32; ++i) m = fmaxf(m, red[i]);
-  __syncthreads();
-  float wsum_part = 0.0f;
-  for (int s = threadIdx.x; s < S; s += kCombineThreads) {
-    const float l = pl[s];
-    const float w = (l == -INFINITY) ? 0.0f : expf(l - m);
-    w_smem[s] = w;
+  for (int k = 0; k < 2; ++k) {
+    const int sidx = threadIdx.x + k * kCombineThreads;
+    const float w = (lse[k] == -INFINITY) ? 0.0f : expf(lse[k] - m);
+    if (sidx < S) w_smem[sidx] = w;
+    wpart += w;
   }
+  // fixed-shape tree sum of the weights (deterministic)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wpart += __shfl_xor_sync(0xffffffffu, wpart, o);
+  if (lane == 0) red[1][wid] = wpart;
   __syncthreads();
-  // every thread sums the weights in the same order (deterministic)
-  for (int s = 0; s < S; ++s) wsum_part += w_smem[s];
+  const float wsum = (red[1][0] + red[1][1]) + (red[1][2] + red[1][3]);
 
-  float acc = 0.0f;
+  // accumulate in four independent chains, summed in a fixed order
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   for (int g0 = 0; g0 < S; g0 += kCombineGroup) {
     if (g0 > 0) {
 #pragma unroll
@@ -71,14 +85,15 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     }
 #pragma unroll
     for (int j = 0; j < kCombineGroup; ++j)
-      if (g0 + j < S) acc = fmaf(w_smem[g0 + j], v[j], acc);
+      if (g0 + j < S) acc[j & 3] = fmaf(w_smem[g0 + j], v[j], acc[j & 3]);
   }
+  const float a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 
-  const bool empty = (m == -INFINITY) || !(wsum_part > 0.0f);
-  const float o = empty ? 0.0f : acc / wsum_part;
+  const bool empty = (m == -INFINITY) || !(wsum > 0.0f);
+  const float o = empty ? 0.0f : a / wsum;
   out[(size_t)row * 512 + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
   if (out_lse != nullptr && blockIdx.y == 0 && threadIdx.x == 0)
-    out_lse[row] = empty ? -INFINITY : m + logf(wsum_part);
+    out_lse[row] = empty ? -INFINITY : m + logf(wsum);
 }
 
 cudaError_t launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
@@ -86,11 +101,20 @@ cudaError_t launch_combine(const float* part_o, const float* part_lse, const int
                            cudaStream_t stream) {
   const int rows = B * q_len * H;
   if (rows == 0) return cudaSuccess;
-  dim3 grid(rows, 512 / kCombineThreads);
-  const size_t smem = sizeof(float) * (size_t)max_splits;
-  combine_kernel<<<grid, kCombineThreads, smem, stream>>>(part_o, part_lse, num_splits, max_splits,
-                                                          q_len * H, out, out_lse);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows, 512 / kCombineThreads);
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = sizeof(float) * (size_t)max_splits;
+  cfg.stream = stream;
+  // programmatic dependent launch: the grid may be scheduled while the
+  // partial kernel before it on the stream is still running
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, part_o, part_lse, num_splits, max_splits,
+                            q_len * H, out, out_lse);
 }
 
 }  // namespace mla

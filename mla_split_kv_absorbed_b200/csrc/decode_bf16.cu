@@ -132,6 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int s = blockIdx.y;
   const int b = blockIdx.z;
   const int QH = args.q_len * args.H;
+  // the merge kernel that follows may be scheduled now; it waits for this
+  // grid's completion before it reads any partial
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---------------------------------------------------------------- split range (step A2)
   const int L = args.seq_lens[b];
