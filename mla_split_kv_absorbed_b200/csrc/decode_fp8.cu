@@ -153,6 +153,96 @@ __device__ __forceinline__ void split8(const float* x, uint2& hi, uint2& lo) {
   lo.y = l[2] | (l[3] << 16);
 }
 
+// Merge of the P CTAs (one cluster) that share a split, each having staged
+// its unnormalised O ([64][512] fp32 at kOffRing), its used max m (sc.m_run)
+// and row sum l (sc.inv_l) in its own shared memory.  With M = max m_k over
+// the pieces that saw a token and l = sum_k l_k 2^(m_k - M), the split's
+// partial is O = sum_k O_k 2^(m_k - M) kv_scale / l and
+// LSE = (M - 7 + log2 l) ln 2, the values one CTA over the whole split
+// produces.  Rank r of the cluster writes rows [r 64/P, (r+1) 64/P).  Every
+// thread of every CTA of the cluster calls this; all distributed shared
+// memory loads of a thread are issued before the first is used.
+template <int P>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs& args, uint8_t* smem, Scratch& sc,
+                                             int64_t row_base, int rows_valid, int s) {
+  constexpr int kRowsPer = kRows / P;
+  constexpr int kIters = (kRowsPer * 128 + kThreads - 1) / kThreads;  // float4 per thread
+  const int tid = threadIdx.x;
+  const uint32_t rank = cluster_ctarank();
+  cluster_sync_all();  // every piece's O, m and l are staged
+  const int n0 = (int)rank * kRowsPer;
+  float* wgt = reinterpret_cast<float*>(smem + kOffPhi);  // [P][64] piece weights (P buffers are free)
+  if (tid < kRowsPer) {
+    const int n = n0 + tid;
+    float mk[P], lk[P];
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      mk[k] = ld_cluster_f32(mapa_shared(smem_u32(&sc.m_run[n]), k));
+      lk[k] = ld_cluster_f32(mapa_shared(smem_u32(&sc.inv_l[n]), k));
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+      if (lk[k] > 0.0f) M = fmaxf(M, mk[k]);
+    float l = 0.0f;
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+      if (lk[k] > 0.0f) l += lk[k] * exp2f(mk[k] - M);
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+      wgt[k * kRows + n] = (lk[k] > 0.0f && l > 0.0f) ? exp2f(mk[k] - M) * args.kv_scale / l : 0.0f;
+    if (n < rows_valid)
+      args.part_lse[(row_base + n) * args.max_splits + s] =
+          l > 0.0f ? (M - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  }
+  __syncthreads();
+  const uint32_t staged = smem_u32(smem + kOffRing);
+  float4 o[kIters][P];
+  float w[kIters][P];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int idx = tid + it * kThreads;
+    const int n = n0 + (idx >> 7);
+    const int q4 = idx & 127;  // dims 4*q4 .. 4*q4+3
+    const bool live = idx < kRowsPer * 128 && n < rows_valid;
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      w[it][k] = live ? wgt[k * kRows + n] : 0.0f;
+      // an empty piece (weight 0) staged nothing: skip its load
+      o[it][k] = w[it][k] != 0.0f
+                     ? ld_cluster_f32x4(mapa_shared(staged + (uint32_t)(n * 512 + 4 * q4) * 4u, k))
+                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int idx = tid + it * kThreads;
+    const int n = n0 + (idx >> 7);
+    const int q4 = idx & 127;
+    if (idx < kRowsPer * 128 && n < rows_valid) {
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+      for (int k = 0; k < P; ++k) {
+        acc.x = fmaf(w[it][k], o[it][k].x, acc.x);
+        acc.y = fmaf(w[it][k], o[it][k].y, acc.y);
+        acc.z = fmaf(w[it][k], o[it][k].z, acc.z);
+        acc.w = fmaf(w[it][k], o[it][k].w, acc.w);
+      }
+      *reinterpret_cast<float4*>(args.part_o + ((row_base + n) * args.max_splits + s) * 512 +
+                                 4 * q4) = acc;
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while a peer still reads its shared memory
+}
+
+__device__ __forceinline__ void merge_pieces(const DecodeArgs& args, uint8_t* smem, Scratch& sc,
+                                             int64_t row_base, int rows_valid, int s) {
+  if (args.pieces == 2)
+    merge_pieces<2>(args, smem, sc, row_base, rows_valid, s);
+  else
+    merge_pieces<4>(args, smem, sc, row_base, rows_valid, s);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fp8_kernel(const DecodeArgs args, const __grid_constant__ CUtensorMap kv_map) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -162,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = tid & 31;
 
   const int g = blockIdx.x;
-  const int s = blockIdx.y;
+  const int s = blockIdx.y / args.pieces;      // split
+  const int piece = blockIdx.y % args.pieces;  // this CTA's run of the split's tiles
   const int b = blockIdx.z;
   const int QH = args.q_len * args.H;
   // the merge kernel that follows may be scheduled now; it waits for this
@@ -173,12 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int L = args.seq_lens[b];
   const int S_b = args.num_splits[b];
   if (S_b < 1 || S_b > args.max_splits) {
-    if (tid == 0 && s == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SPLITS);
+    if (tid == 0 && blockIdx.y == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SPLITS);
     return;
   }
   if (s >= S_b) return;
   if (L < args.q_len || (int64_t)L > (int64_t)args.max_pages * 64) {
-    if (tid == 0 && s == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SEQLEN);
+    if (tid == 0 && blockIdx.y == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SEQLEN);
     return;
   }
   const int n_pages = (L + 63) / 64;
@@ -190,24 +281,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q_min = r0 / args.H;
   const int q_max = (r0 + rows_valid - 1) / args.H;
   const int vis_base = L - args.q_len + 1;  // visible length of q = 0
-  const int t0 = p0 * 64;
-  const int t1 = min(p1 * 64, vis_base + q_max);
-  const int t_all = min(t1, vis_base + q_min);  // every column sees every token < t_all
+  const int t0s = p0 * 64;                         // the split's tokens [t0s, t1s)
+  const int t1s = min(p1 * 64, vis_base + q_max);
   const int64_t row_base = (int64_t)b * QH + r0;
 
-  if (t1 <= t0) {  // empty split for every row of the group
-    for (int i = tid; i < rows_valid * 512; i += kThreads) {
-      const int n = i >> 9;
-      args.part_o[((row_base + n) * args.max_splits + s) * 512 + (i & 511)] = 0.0f;
+  if (t1s <= t0s) {  // empty split for every row of the group
+    if (piece == 0) {
+      for (int i = tid; i < rows_valid * 512; i += kThreads) {
+        const int n = i >> 9;
+        args.part_o[((row_base + n) * args.max_splits + s) * 512 + (i & 511)] = 0.0f;
+      }
+      if (tid < rows_valid) args.part_lse[(row_base + tid) * args.max_splits + s] = -INFINITY;
     }
-    if (tid < rows_valid) args.part_lse[(row_base + tid) * args.max_splits + s] = -INFINITY;
     return;
   }
-  const int T = (t1 - t0 + kTile - 1) / kTile;
+  // this CTA's run: tiles [tile0, tile0 + T) of the split's Ts tiles
+  const int Ts = (t1s - t0s + kTile - 1) / kTile;
+  const int per = (Ts + args.pieces - 1) / args.pieces;
+  const int tile0 = min(piece * per, Ts);
+  const int T = min(per, Ts - tile0);  // 0 only for a trailing piece of a short split
+  const int pg0 = p0 + 2 * tile0;      // block-table index of the run's first page
+  const int t0 = t0s + tile0 * kTile;
+  const int t1 = min(t1s, t0 + T * kTile);
+  const int t_all = min(t1, vis_base + q_min);  // every column sees every token < t_all
 
   // ---------------------------------------------------------------- setup
-  if ((smem_u32(smem) & 1023u) != 0) {
+  if ((smem_u32(smem) & 1023u) != 0) {  // same for every CTA of the grid
     if (tid == 0) set_error(args.dev_error, MLA_DEVERR_SMEM_ALIGN);
+    return;
+  }
+  if (T == 0) {
+    // no tiles in this piece: it joins the cluster merge with an empty result
+    if (tid < 64) {
+      sc.m_run[tid] = -INFINITY;
+      sc.inv_l[tid] = 0.0f;
+    }
+    __syncthreads();
+    merge_pieces(args, smem, sc, row_base, rows_valid, s);
     return;
   }
   if (tid == 0) {
@@ -258,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // skipped here and reported by the load path
     auto prefetch_tile = [&](int i) {
       const int tok0 = t0 + i * kTile;
-      const int pa = bt[p0 + 2 * i];
+      const int pa = bt[pg0 + 2 * i];
       const bool want_b = tok0 + 64 < t1;
-      const int pb = want_b ? bt[p0 + 2 * i + 1] : -1;
+      const int pb = want_b ? bt[pg0 + 2 * i + 1] : -1;
       if (pa >= 0 && (int64_t)pa < args.num_pages)
         bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pa * kPageBytes, kPageBytes);
       if (want_b && pb >= 0 && (int64_t)pb < args.num_pages)
@@ -275,9 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < T && ok; ++i) {
       if (i + 3 < T) prefetch_tile(i + 3);
       const int tok0 = t0 + i * kTile;
-      const int pa = bt[p0 + 2 * i];
+      const int pa = bt[pg0 + 2 * i];
       const bool want_b = tok0 + 64 < t1;
-      const int pb = want_b ? bt[p0 + 2 * i + 1] : 0;
+      const int pb = want_b ? bt[pg0 + 2 * i + 1] : 0;
       const bool la = pa >= 0 && (int64_t)pa < args.num_pages;
       const bool lb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
       if (lane == 0 && (!la || (want_b && !lb))) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
@@ -612,10 +722,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = (sc.warp_max[wg][0][lane] + sc.warp_max[wg][1][lane]) +
                         (sc.warp_max[wg][2][lane] + sc.warp_max[wg][3][lane]);
         const bool nonempty = ok && l > 0.0f;
-        sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
-        if (n < rows_valid)
-          args.part_lse[(row_base + n) * args.max_splits + s] =
-              nonempty ? (sc.m_run[n] - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        if (args.pieces == 1) {
+          sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
+          if (n < rows_valid)
+            args.part_lse[(row_base + n) * args.max_splits + s] =
+                nonempty ? (sc.m_run[n] - kPShift + log2f(l)) * 0.69314718055994530942f
+                         : -INFINITY;
+        } else {
+          sc.inv_l[n] = nonempty ? l : 0.0f;  // raw row sum, merged across the cluster
+        }
       }
     }
     named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
@@ -678,15 +793,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
       float* po = args.part_o + (row_base * args.max_splits + s) * 512;
       const int64_t row_stride = (int64_t)args.max_splits * 512;
+      float* staged = reinterpret_cast<float*>(smem + kOffRing);  // [64][512], ring is free
 #pragma unroll 1
       for (int c = ewg; c < 16; c += 5) {
         const int j = c >> 2, grp = c & 3;
         float v[16];
         tmem_ld16(t_lane + 256 + 64 * j + 16 * grp, v);
+        if (args.pieces == 1) {
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          const int n = grp * 16 + cc;
-          if (n < rows_valid) po[n * row_stride + 128 * j + d_lane] = v[cc] * sc.inv_l[n];
+          for (int cc = 0; cc < 16; ++cc) {
+            const int n = grp * 16 + cc;
+            if (n < rows_valid) po[n * row_stride + 128 * j + d_lane] = v[cc] * sc.inv_l[n];
+          }
+        } else {
+          // unnormalised O, merged across the cluster below
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) staged[(grp * 16 + cc) * 512 + 128 * j + d_lane] = v[cc];
         }
       }
     }
@@ -699,6 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (args.pieces > 1) merge_pieces(args, smem, sc, row_base, rows_valid, s);
 }
 
 }  // namespace fp8k
@@ -713,9 +836,26 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cu
     configured = true;
   }
   const int groups = (a.q_len * a.H + fp8k::kRows - 1) / fp8k::kRows;
-  dim3 grid(groups, a.max_splits, a.B);
-  fp8k::decode_fp8_kernel<<<grid, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map);
-  return cudaGetLastError();
+  if (a.pieces == 1) {
+    fp8k::decode_fp8_kernel<<<dim3(groups, a.max_splits, a.B), fp8k::kThreads, fp8k::kSmemBytes,
+                              stream>>>(a, kv_map);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(groups, a.max_splits * a.pieces, a.B);
+  cfg.blockDim = dim3(fp8k::kThreads);
+  cfg.dynamicSmemBytes = fp8k::kSmemBytes;
+  cfg.stream = stream;
+  // the pieces of one split form a cluster (they merge through distributed
+  // shared memory)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)a.pieces;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fp8k::decode_fp8_kernel, a, kv_map);
 }
 
 }  // namespace mla

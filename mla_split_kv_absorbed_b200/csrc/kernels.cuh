@@ -32,6 +32,7 @@ struct DecodeArgs {
   int H;
   float qk_scale_log2;  // softmax_scale * kv_scale * log2(e)
   float kv_scale;
+  int pieces;           // CTAs per split (a cluster), each over a contiguous run of its tiles
 };
 
 // FP8 E4M3 cache: kv_map is a 3-D tiled TMA map over kv_pages viewed as

@@ -139,6 +139,16 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   a.H = H;
   a.qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
   a.kv_scale = kv_scale;
+  // When the (group, split, request) grid fills at most half of the SMs, each
+  // split is cut into 2 or 4 contiguous runs of tiles processed by a cluster
+  // of CTAs that merges its results on chip (FP8 path); the partial per split
+  // is unchanged.
+  a.pieces = 1;
+  if (kv_dtype == MLA_KV_FP8_E4M3) {
+    const long long units = (long long)((q_len * H + 63) / 64) * max_splits * B;
+    const int sms = num_sms_cached();
+    while (a.pieces < 4 && units * a.pieces * 2 <= sms) a.pieces *= 2;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, s)
                                                : mla::launch_decode_bf16(a, map, s));

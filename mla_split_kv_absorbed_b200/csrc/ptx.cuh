@@ -113,6 +113,39 @@ __device__ __forceinline__ void tma_prefetch_l2_3d_elect(const CUtensorMap* map,
       "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// ---- thread-block clusters: rank, distributed shared memory, cluster barrier
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared::cta offset in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+// every thread of every CTA of the cluster; release/acquire orders shared
+// memory writes before it against reads after it, cluster-wide
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Untiled bulk L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned
 // global address; one elected lane of the (converged) warp issues it.
 __device__ __forceinline__ void bulk_prefetch_l2_elect(const void* gaddr, uint32_t bytes) {
