@@ -171,6 +171,18 @@ MLA_API int mla_decode_noalloc(const uint16_t* q_nope, const uint16_t* q_rope,
 MLA_API int mla_choose_splits(const int32_t* seq_lens_host, int B, int q_len, int H,
                       int num_sms, int max_splits, int32_t* out_host);
 
+/* ---------------------------------------------------------------------------
+ * mla_debug_inject_stall: a test hook for the failure path; the pages have no
+ * counterpart.  While enabled (enable != 0), every FP8 mla_decode_partial
+ * launch leaves the first KV load of its first CTA (first tile, first latent
+ * pair) unissued, so the waits on that load run out: after the 2 s bound the
+ * kernel sets MLA_DEVERR_TIMEOUT in dev_error, all of its warps leave their
+ * loops, it frees its tensor memory and returns.  Nothing traps or faults and
+ * the CUDA context stays usable; the outputs of such a launch are undefined.
+ * Returns the previous setting.  Process-wide; not for production use.
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_debug_inject_stall(int enable);
+
 /* Static, human-readable name of a status code. */
 MLA_API const char* mla_status_string(int status);
 

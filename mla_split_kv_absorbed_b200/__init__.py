@@ -71,6 +71,8 @@ def _load_lib():
     lib.mla_choose_splits.restype = i32
     lib.mla_status_string.argtypes = [i32]
     lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_debug_inject_stall.argtypes = [i32]
+    lib.mla_debug_inject_stall.restype = i32
     return lib
 
 
@@ -181,6 +183,13 @@ def mla_choose_splits(seq_lens_host, q_len: int, H: int, num_sms: int, max_split
 
 def mla_status_string(status: int) -> str:
     return status_string(status)
+
+
+def mla_debug_inject_stall(enable: bool) -> bool:
+    """Test hook: while enabled, FP8 partial launches leave one KV load of
+    their first CTA unissued, so its bounded waits run out and the kernel
+    reports MLA_DEVERR_TIMEOUT.  Returns the previous setting."""
+    return bool(_lib.mla_debug_inject_stall(1 if enable else 0))
 
 
 def decode(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits, max_splits,

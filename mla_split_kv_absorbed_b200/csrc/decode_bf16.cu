@@ -58,8 +58,8 @@ constexpr int kBarPEmpty = 13;
 constexpr int kBarOReady = 14;
 constexpr int kBarPvDone = 15;
 constexpr int kBarQReady = 16;
-constexpr int kBarAlphaFull = 17;
-constexpr int kBarDrain = 18;
+constexpr int kBarAlphaFull = 17;  // 2: per tile parity (the softmax groups may be a tile apart)
+constexpr int kBarDrain = 19;
 
 struct Scratch {
   uint64_t bars[24];
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sc.bars[kBarOReady], 128);
     mbar_init(&sc.bars[kBarPvDone], 1);
     mbar_init(&sc.bars[kBarQReady], 8);
-    mbar_init(&sc.bars[kBarAlphaFull], 2);
+    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarAlphaFull + i], 2);
     mbar_init(&sc.bars[kBarDrain], 1);
     sc.abort = 0;
     fence_barrier_init();
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) sc.changed[i & 1][wg] = mask;
       }
       named_bar_sync(bar_id, 128);
-      if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull]);
+      if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
       const float4* m4 = reinterpret_cast<const float4*>(sc.m_run + col0);
       const float4* a4 = reinterpret_cast<const float4*>(sc.alpha[i & 1] + col0);
       uint32_t pk[16];
@@ -496,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int i = 0; i < T; ++i) {
       if (warp == 12 && lane == 0) {
-        mbar_wait(&bars[kBarAlphaFull], i & 1, abort_flag);
+        mbar_wait(&bars[kBarAlphaFull + (i & 1)], (i >> 1) & 1, abort_flag);
         if (i >= 1) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
       }
       if (named_bar_or(3, 128, *abort_flag != 0)) {

@@ -97,8 +97,8 @@ constexpr int kBarPEmpty = 23;
 constexpr int kBarOReady = 24;
 constexpr int kBarPvDone = 25;
 constexpr int kBarQReady = 26;
-constexpr int kBarAlphaFull = 27;
-constexpr int kBarDrain = 28;
+constexpr int kBarAlphaFull = 27;  // 2: per tile parity (the softmax groups may be a tile apart)
+constexpr int kBarDrain = 29;
 
 struct Scratch {
   uint64_t bars[32];
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sc.bars[kBarOReady], 128);
     mbar_init(&sc.bars[kBarPvDone], 1);
     mbar_init(&sc.bars[kBarQReady], 4 * kSoftGroups);
-    mbar_init(&sc.bars[kBarAlphaFull], kSoftGroups);
+    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarAlphaFull + i], kSoftGroups);
     mbar_init(&sc.bars[kBarDrain], 1);
     sc.abort = 0;
     fence_barrier_init();
@@ -400,6 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
         }
         uint64_t* full = &bars[kBarNopeFull + slot];
+        if (args.inject_stall && i == 0 && j == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+            blockIdx.z == 0)
+          continue;  // test hook: this slot is never armed, so its waits run out
         mbar_arrive_expect_tx_elect(full, 2 * bytes_chunk);
         armed[slot] = true;
         last_nope_parity[slot] = (i >> 1) & 1;
@@ -664,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) sc.changed[i & 1][wg] = mask;
       }
       named_bar_sync(bar_id, 128);
-      if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull]);
+      if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
       const float4* m4 = reinterpret_cast<const float4*>(sc.m_run + col0);
       const float4* a4 = reinterpret_cast<const float4*>(sc.alpha[i & 1] + col0);
       uint2 phi[kCols / 8], plo[kCols / 8];
@@ -741,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int i = 0; i < T; ++i) {
       if (wq == 0 && lane == 0) {
-        mbar_wait(&bars[kBarAlphaFull], i & 1, abort_flag);
+        mbar_wait(&bars[kBarAlphaFull + (i & 1)], (i >> 1) & 1, abort_flag);
         if (i >= 1) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
       }
       if (named_bar_or(5, 128, *abort_flag != 0)) {

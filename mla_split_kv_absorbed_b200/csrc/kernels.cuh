@@ -33,6 +33,7 @@ struct DecodeArgs {
   float qk_scale_log2;  // softmax_scale * kv_scale * log2(e)
   float kv_scale;
   int pieces;           // CTAs per split (a cluster), each over a contiguous run of its tiles
+  int inject_stall;     // test hook: leave the first load of CTA (0, 0, 0) unissued
 };
 
 // FP8 E4M3 cache: kv_map is a 3-D tiled TMA map over kv_pages viewed as

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -12,6 +13,8 @@
 #include "mla.h"
 
 namespace {
+
+std::atomic<int> g_inject_stall{0};  // mla_debug_inject_stall
 
 constexpr int kPage = 64;
 constexpr int kRow = 576;
@@ -143,6 +146,7 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   // split is cut into 2 or 4 contiguous runs of tiles processed by a cluster
   // of CTAs that merges its results on chip (FP8 path); the partial per split
   // is unchanged.
+  a.inject_stall = g_inject_stall.load(std::memory_order_relaxed);
   a.pieces = 1;
   if (kv_dtype == MLA_KV_FP8_E4M3) {
     const long long units = (long long)((q_len * H + 63) / 64) * max_splits * B;
@@ -200,6 +204,10 @@ const char* mla_status_string(int status) {
     case MLA_ERR_SCRATCH_LIMIT: return "MLA_ERR_SCRATCH_LIMIT";
     default: return "MLA_ERR_UNKNOWN";
   }
+}
+
+int mla_debug_inject_stall(int enable) {
+  return g_inject_stall.exchange(enable != 0 ? 1 : 0, std::memory_order_relaxed);
 }
 
 }  // extern "C"

@@ -1,0 +1,52 @@
+"""Failure detection on the GPU without a fault.
+
+Every wait in the partial kernel is bounded (2 s, %globaltimer).  The library's
+test hook leaves one KV load of the first CTA unissued, so the waits on it
+run out: the kernel must report MLA_DEVERR_TIMEOUT through the caller's error
+word, return within a bounded time, and leave the CUDA context usable (the next
+decode matches the oracle).  No trap, no device assert, no bad address.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import assert_attention_close, make_case, oracle_rows, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+# 128 splits of one page each: the grid fills more than half of the SMs, so
+# every split is one CTA (no cluster), and CTA (0, 0, 0) is split 0.
+CASE = ("b1_128k_fp8", dict(seq_lens=[8192], splits=128))
+
+
+def test_stalled_load_times_out_and_context_survives():
+    import mla_split_kv_absorbed_b200 as m
+    c = make_case(CASE[0], **CASE[1])
+    w = c.w
+    part_o, part_lse = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    prev = m.mla_debug_inject_stall(True)
+    try:
+        t0 = time.perf_counter()
+        m.mla_decode_partial(c.dev["q_nope"], c.dev["q_rope"], c.kv_dev, w.kv_scale,
+                             c.dev["block_table"], c.dev["seq_lens"], c.dev["num_splits"],
+                             w.max_splits, w.softmax_scale, part_o, part_lse, err)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        m.mla_debug_inject_stall(prev)
+    word = int(err.item())
+    print(f"[failure] error word {word:#x} after {elapsed:.2f} s")
+    assert word & m.DEVERR_TIMEOUT, f"timeout not reported (error word {word:#x})"
+    assert elapsed < 30.0, f"kernel took {elapsed:.1f} s to give up"
+
+    # the context is intact: the same decode without the hook is correct
+    out, lse, _, _, err2 = run_gpu(c)
+    assert err2 == 0
+    rows = np.arange(w.B * w.q_len * w.H)
+    o_ref, l_ref = oracle_rows(c, rows)
+    assert_attention_close(out.float().cpu().numpy().reshape(-1, 512),
+                           lse.cpu().numpy().reshape(-1), o_ref, l_ref, what="after timeout")
