@@ -106,6 +106,33 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+KERNEL_SOURCES = {
+    "decode_fp8_kernel": ["decode_fp8.cu", "ptx.cuh", "kernels.cuh"],
+    "decode_bf16_kernel": ["decode_bf16.cu", "ptx.cuh", "kernels.cuh"],
+}
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from profiles/traffic.txt, if it was measured on
+    the kernel sources as they are now (SHA-256 match), else None."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(here, "mla_split_kv_absorbed_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    try:
+        with open(os.path.join(here, "profiles", "traffic.txt")) as fh:
+            for line in fh:
+                parts = line.split()
+                if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel \
+                        and parts[1] == workload and parts[2] == h.hexdigest():
+                    return int(parts[3])
+    except OSError:
+        pass
+    return None
+
+
 def setup_workload(name, device):
     import torch
     import mla_split_kv_absorbed_b200 as m
@@ -354,6 +381,7 @@ def main():
         cpu = cpu_baseline(w, host_codes(w, kv))
 
     achieved = w.kv_bytes / t_partial / 1e9
+    kernel_name = "decode_fp8_kernel" if w.spec.kv_dtype == "fp8" else "decode_bf16_kernel"
     line = {
         "metric": METRIC,
         "value": value,
@@ -375,9 +403,10 @@ def main():
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "kernel": "decode_fp8_kernel" if w.spec.kv_dtype == "fp8" else "decode_bf16_kernel",
-                     "kernel_us": t_partial * 1e6, "peak_kind": peak_kind},
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(kernel_name, args.workload),
+                     "algorithmic_bytes": w.kv_bytes,
+                     "kernel": kernel_name, "kernel_us": t_partial * 1e6, "peak_kind": peak_kind},
         "e2e": {"value": ws * w.kv_bytes / e2e_t / 1e9, "unit": "GB/s", "us_per_step": e2e_t * 1e6,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
