@@ -36,8 +36,10 @@
 //
 // Online softmax (log2 domain, scores pre-multiplied by log2 e), with a lazy
 // running max: the max m used for a row only moves when a tile's max exceeds
-// it by more than 1 (a factor of 2), so p' stays <= 2^8 and rescaling of the
-// O^T columns and row sums (by 2^(m_old - m_new)) is rare.
+// it by more than 1.75 (log2 units), so p' stays <= 2^8.75 < 448, the E4M3
+// maximum, and rescaling of the O^T columns and row sums (by
+// 2^(m_old - m_new)) is rare.  A tile whose max moved nowhere does not wait
+// for the previous tile's PV before its own PV is released.
 //
 // Warp roles (768 threads):
 //   warp 0        TMA producer: pages -> 64-byte-swizzled chunks, plus L2
@@ -75,7 +77,7 @@ constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
 constexpr uint32_t kPageBytes = 64 * 576;  // one page of the pool
 constexpr int kRingPairs = 8;       // two tiles of latent dims in flight
 constexpr float kPShift = 7.0f;     // log2 of the factor carried by the softmax weights
-constexpr float kLazy = 1.0f;       // the used max moves only when exceeded by more than this
+constexpr float kLazy = 1.75f;       // the used max moves only when exceeded by more than this
 
 constexpr int kOffQ = 0;                                 // 9 chunks, rows hi 0-63 | lo 64-127
 constexpr int kOffRing = kOffQ + 9 * kChunk;             // 73728
@@ -94,11 +96,11 @@ constexpr int kBarSFull = 18;      // 2
 constexpr int kBarSEmpty = 20;     // 2
 constexpr int kBarPFull = 22;
 constexpr int kBarPEmpty = 23;
-constexpr int kBarOReady = 24;
-constexpr int kBarPvDone = 25;
-constexpr int kBarQReady = 26;
-constexpr int kBarAlphaFull = 27;  // 2: per tile parity (the softmax groups may be a tile apart)
-constexpr int kBarDrain = 29;
+constexpr int kBarOReady = 24;     // 2: per tile parity (the rescale loop may run a tile ahead)
+constexpr int kBarPvDone = 26;
+constexpr int kBarQReady = 27;
+constexpr int kBarAlphaFull = 28;  // 2: per tile parity (the softmax groups may be a tile apart)
+constexpr int kBarDrain = 30;
 
 struct Scratch {
   uint64_t bars[32];
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sc.bars[kBarPFull], kSoftThreads);
     mbar_init(&sc.bars[kBarPEmpty], 1);
-    mbar_init(&sc.bars[kBarOReady], 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarOReady + i], 128);
     mbar_init(&sc.bars[kBarPvDone], 1);
     mbar_init(&sc.bars[kBarQReady], 4 * kSoftGroups);
     for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarAlphaFull + i], kSoftGroups);
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // ---------------- O^T += V(np)^T . (P_hi + P_lo)
-      if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady, np & 1)) {
+      if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady + (np & 1), (np >> 1) & 1)) {
         tc_fence_after();
         const uint32_t slot0 = (np & 1) * 4 * kPair;
         // block by block, so each latent pair can be refilled as soon as its
@@ -681,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int j = 8 * q8 + k;
-          // weights carry a 2^7 factor: p' = 2^(s - m + 7) <= 2^8
+          // weights carry a 2^7 factor: p' = 2^(s - m + 7) <= 2^8.75
           pv[k] = (sv[j] == -INFINITY) ? 0.0f : ex2_approx(sv[j] - mm[k] + kPShift);
           l_part[j] = fmaf(l_part[j], al[k], pv[k]);
         }
@@ -739,47 +741,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
   } else if (warp >= 4 + 4 * kSoftGroups) {
     // ============================================================ O^T rescale between tiles
+    // The O-ready barriers are per tile parity because this loop may run one
+    // tile ahead of the PV issue, but never two: tile i + 2 needs the ring
+    // slots that PV(i) frees, and so its max and alpha.
     const int wq = warp & 3;            // thread = latent dim wq * 32 + lane of a block
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     bool ok = true;
     for (int i = 0; i < T; ++i) {
-      if (wq == 0 && lane == 0) {
-        mbar_wait(&bars[kBarAlphaFull + (i & 1)], (i >> 1) & 1, abort_flag);
-        if (i >= 1) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
-      }
+      if (wq == 0 && lane == 0) mbar_wait(&bars[kBarAlphaFull + (i & 1)], (i >> 1) & 1, abort_flag);
       if (named_bar_or(5, 128, *abort_flag != 0)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      if (i >= 1) {
-        const uint32_t ch0 = sc.changed[i & 1][0], ch1 = sc.changed[i & 1][1];
-        const uint32_t ch2 = sc.changed[i & 1][2], ch3 = sc.changed[i & 1][3];
-        if ((ch0 | ch1 | ch2 | ch3) != 0) {
+      const uint32_t ch0 = i >= 1 ? sc.changed[i & 1][0] : 0u, ch1 = i >= 1 ? sc.changed[i & 1][1] : 0u;
+      const uint32_t ch2 = i >= 1 ? sc.changed[i & 1][2] : 0u, ch3 = i >= 1 ? sc.changed[i & 1][3] : 0u;
+      if ((ch0 | ch1 | ch2 | ch3) != 0) {
+        // some column's max moved: O^T is rescaled once PV of the previous tile is done
+        if (wq == 0 && lane == 0) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
+        named_bar_sync(5, 128);
+        tc_fence_after();
 #pragma unroll 1
-          for (int grp = 0; grp < 4; ++grp) {  // grp = softmax group = 16 columns
-            const uint32_t bits = grp == 0 ? ch0 : grp == 1 ? ch1 : grp == 2 ? ch2 : ch3;
-            if (bits == 0) continue;
-            float a[16];
+        for (int grp = 0; grp < 4; ++grp) {  // grp = softmax group = 16 columns
+          const uint32_t bits = grp == 0 ? ch0 : grp == 1 ? ch1 : grp == 2 ? ch2 : ch3;
+          if (bits == 0) continue;
+          float a[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) a[c] = sc.alpha[i & 1][grp * 16 + c];
+          for (int c = 0; c < 16; ++c) a[c] = sc.alpha[i & 1][grp * 16 + c];
 #pragma unroll 1
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t ta = t_lane + 256 + 64 * j + 16 * grp;
-              float v[16];
-              tmem_ld16(ta, v);
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t ta = t_lane + 256 + 64 * j + 16 * grp;
+            float v[16];
+            tmem_ld16(ta, v);
 #pragma unroll
-              for (int c = 0; c < 16; ++c) v[c] *= a[c];
-              tmem_st16(ta, v);
-            }
+            for (int c = 0; c < 16; ++c) v[c] *= a[c];
+            tmem_st16(ta, v);
           }
-          tmem_wait_st();
         }
+        tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&bars[kBarOReady]);
+      mbar_arrive(&bars[kBarOReady + (i & 1)]);
     }
-    if (ok && wq == 0 && lane == 0) mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
+    // This loop may have run a tile ahead of PV, so the barrier can still be
+    // one phase short of tile T-2: wait for that phase first, or the parity
+    // test for T-1 would match the older phase T-3.
+    if (ok && wq == 0 && lane == 0) {
+      if (T >= 2) mbar_wait(&bars[kBarPvDone], (T - 2) & 1, abort_flag);
+      mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
+    }
     named_bar_sync(5, 128);
     tc_fence_before();
     named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
