@@ -237,9 +237,9 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs& args, uint8_t* sm
   cluster_sync_all();  // no CTA leaves while a peer still reads its shared memory
 }
 
-__device__ __forceinline__ void merge_pieces(const DecodeArgs& args, uint8_t* smem, Scratch& sc,
-                                             int64_t row_base, int rows_valid, int s) {
-  if (args.pieces == 2)
+__device__ __forceinline__ void merge_pieces(int npieces, const DecodeArgs& args, uint8_t* smem,
+                                             Scratch& sc, int64_t row_base, int rows_valid, int s) {
+  if (npieces == 2)
     merge_pieces<2>(args, smem, sc, row_base, rows_valid, s);
   else
     merge_pieces<4>(args, smem, sc, row_base, rows_valid, s);
@@ -253,25 +253,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  const int g = blockIdx.x;
-  const int s = blockIdx.y / args.pieces;      // split
-  const int piece = blockIdx.y % args.pieces;  // this CTA's run of the split's tiles
-  const int b = blockIdx.z;
   const int QH = args.q_len * args.H;
   // the merge kernel that follows may be scheduled now; it waits for this
   // grid's completion before it reads any partial
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+  // unit (query-row group g, split s, request b) and this CTA's piece of it
+  int unit, piece = 0, npieces = 1;
+  if ((int)blockIdx.x < args.split_from) {
+    unit = blockIdx.x;
+  } else if ((int)blockIdx.x < args.split_from + args.pad) {
+    return;  // idle: only aligns the clusters of the split units
+  } else {
+    const int j = (int)blockIdx.x - args.split_from - args.pad;
+    unit = args.split_from + j / args.pieces;
+    piece = j % args.pieces;  // this CTA's run of the split's tiles
+    npieces = args.pieces;
+  }
+  const int g = unit % args.groups;
+  const int s = (unit / args.groups) % args.max_splits;
+  const int b = unit / (args.groups * args.max_splits);
+
   // ---------------------------------------------------------------- split range (step A2)
   const int L = args.seq_lens[b];
   const int S_b = args.num_splits[b];
   if (S_b < 1 || S_b > args.max_splits) {
-    if (tid == 0 && blockIdx.y == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SPLITS);
+    if (tid == 0 && s == 0 && g == 0 && piece == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SPLITS);
     return;
   }
   if (s >= S_b) return;
   if (L < args.q_len || (int64_t)L > (int64_t)args.max_pages * 64) {
-    if (tid == 0 && blockIdx.y == 0 && g == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SEQLEN);
+    if (tid == 0 && s == 0 && g == 0 && piece == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SEQLEN);
     return;
   }
   const int n_pages = (L + 63) / 64;
@@ -299,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // this CTA's run: tiles [tile0, tile0 + T) of the split's Ts tiles
   const int Ts = (t1s - t0s + kTile - 1) / kTile;
-  const int per = (Ts + args.pieces - 1) / args.pieces;
+  const int per = (Ts + npieces - 1) / npieces;
   const int tile0 = min(piece * per, Ts);
   const int T = min(per, Ts - tile0);  // 0 only for a trailing piece of a short split
   const int pg0 = p0 + 2 * tile0;      // block-table index of the run's first page
@@ -319,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sc.inv_l[tid] = 0.0f;
     }
     __syncthreads();
-    merge_pieces(args, smem, sc, row_base, rows_valid, s);
+    merge_pieces(npieces, args, smem, sc, row_base, rows_valid, s);
     return;
   }
   if (tid == 0) {
@@ -402,8 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
         }
         uint64_t* full = &bars[kBarNopeFull + slot];
-        if (args.inject_stall && i == 0 && j == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
-            blockIdx.z == 0)
+        if (args.inject_stall && i == 0 && j == 0 && blockIdx.x == 0)
           continue;  // test hook: this slot is never armed, so its waits run out
         mbar_arrive_expect_tx_elect(full, 2 * bytes_chunk);
         armed[slot] = true;
@@ -727,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = (sc.warp_max[wg][0][lane] + sc.warp_max[wg][1][lane]) +
                         (sc.warp_max[wg][2][lane] + sc.warp_max[wg][3][lane]);
         const bool nonempty = ok && l > 0.0f;
-        if (args.pieces == 1) {
+        if (npieces == 1) {
           sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
           if (n < rows_valid)
             args.part_lse[(row_base + n) * args.max_splits + s] =
@@ -811,7 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = c >> 2, grp = c & 3;
         float v[16];
         tmem_ld16(t_lane + 256 + 64 * j + 16 * grp, v);
-        if (args.pieces == 1) {
+        if (npieces == 1) {
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc) {
             const int n = grp * 16 + cc;
@@ -833,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (args.pieces > 1) merge_pieces(args, smem, sc, row_base, rows_valid, s);
+  if (npieces > 1) merge_pieces(npieces, args, smem, sc, row_base, rows_valid, s);
 }
 
 }  // namespace fp8k
@@ -847,23 +858,24 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cu
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int groups = (a.q_len * a.H + fp8k::kRows - 1) / fp8k::kRows;
+  const long long units = (long long)a.groups * a.max_splits * a.B;
+  const long long ctas = a.split_from + a.pad + (units - a.split_from) * a.pieces;
   if (a.pieces == 1) {
-    fp8k::decode_fp8_kernel<<<dim3(groups, a.max_splits, a.B), fp8k::kThreads, fp8k::kSmemBytes,
-                              stream>>>(a, kv_map);
+    fp8k::decode_fp8_kernel<<<(unsigned)ctas, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(groups, a.max_splits * a.pieces, a.B);
+  cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(fp8k::kThreads);
   cfg.dynamicSmemBytes = fp8k::kSmemBytes;
   cfg.stream = stream;
   // the pieces of one split form a cluster (they merge through distributed
-  // shared memory)
+  // shared memory); the one-CTA units are paired into clusters that do not
+  // interact
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = (unsigned)a.pieces;
+  attr[0].val.clusterDim.x = (unsigned)a.pieces;
+  attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;

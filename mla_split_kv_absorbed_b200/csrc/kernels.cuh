@@ -32,7 +32,15 @@ struct DecodeArgs {
   int H;
   float qk_scale_log2;  // softmax_scale * kv_scale * log2(e)
   float kv_scale;
-  int pieces;           // CTAs per split (a cluster), each over a contiguous run of its tiles
+  // FP8 grid, one dimension: units are (query-row group, split, request)
+  // triples, unit = g + groups * (s + max_splits * b).  Units below split_from
+  // run one CTA each; then come `pad` idle CTAs (cluster alignment); every
+  // later unit runs `pieces` CTAs, one cluster, each over a contiguous run of
+  // the split's tiles, merged on chip.
+  int groups;
+  int split_from;
+  int pad;
+  int pieces;
   int inject_stall;     // test hook: leave the first load of CTA (0, 0, 0) unissued
 };
 

@@ -124,7 +124,7 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   int st = make_kv_map(&map, kv_pages, kv_dtype, num_pages);
   if (st != MLA_OK) return st;
 
-  mla::DecodeArgs a;
+  mla::DecodeArgs a = {};
   a.q_nope = q_nope;
   a.q_rope = q_rope;
   a.kv_pages = static_cast<const uint8_t*>(kv_pages);
@@ -142,16 +142,30 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   a.H = H;
   a.qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
   a.kv_scale = kv_scale;
-  // When the (group, split, request) grid fills at most half of the SMs, each
-  // split is cut into 2 or 4 contiguous runs of tiles processed by a cluster
-  // of CTAs that merges its results on chip (FP8 path); the partial per split
-  // is unchanged.
   a.inject_stall = g_inject_stall.load(std::memory_order_relaxed);
+  // FP8 path: when the (group, split, request) units fill at most half of the
+  // SMs, every split is cut into 2 or 4 runs of tiles, one CTA each, merged
+  // on chip by its cluster; when they fill several waves and the last wave is
+  // at most half full, only the units of that last wave are cut in two.  The
+  // partial per split is the same either way.
+  a.groups = (q_len * H + 63) / 64;
+  const long long units = (long long)a.groups * max_splits * B;
   a.pieces = 1;
+  a.split_from = (int)units;
+  a.pad = 0;
   if (kv_dtype == MLA_KV_FP8_E4M3) {
-    const long long units = (long long)((q_len * H + 63) / 64) * max_splits * B;
     const int sms = num_sms_cached();
-    while (a.pieces < 4 && units * a.pieces * 2 <= sms) a.pieces *= 2;
+    if (units * 2 <= sms) {
+      while (a.pieces < 4 && units * a.pieces * 2 <= sms) a.pieces *= 2;
+      a.split_from = 0;
+    } else if (units > sms) {
+      const long long tail = units % sms;
+      if (tail > 0 && tail * 2 <= sms) {
+        a.pieces = 2;
+        a.split_from = (int)(units - tail);
+      }
+    }
+    if (a.pieces > 1) a.pad = (a.pieces - a.split_from % a.pieces) % a.pieces;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, s)

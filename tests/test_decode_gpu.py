@@ -3,7 +3,9 @@
 Small cases span several 128-token tiles, ragged page tails, empty splits,
 q_len 1-4 with causal masking (one query position per row group, and four
 positions inside one group), 16 to 128 heads and NaN-poisoned pages around
-the visible range.  The full-size cases run the benchmark workloads in the
+the visible range.  Small grids exercise the cluster path in which every
+split is cut across 2 or 4 CTAs; one case has a partly filled last wave whose
+units alone are cut.  The full-size cases run the benchmark workloads in the
 benchmark's launch configuration and compare sampled rows.
 """
 import numpy as np
@@ -29,6 +31,9 @@ SMALL = [
     ("b16_128k_fp8", dict(seq_lens=[3000], splits=4, H=128)),
     ("b16_128k_fp8", dict(seq_lens=[1024], splits=4, H=16)),
     ("b16_128k_fp8", dict(seq_lens=[1500, 900], splits=2, H=32, q_len=2)),
+    # 5 x 32 = 160 (group, split) units on 148 SMs: the last, partly filled
+    # wave (12 units) is cut into 2-CTA clusters; short splits give empty pieces
+    ("b16_128k_fp8", dict(seq_lens=[5000, 3000, 64, 4100, 777], splits=32)),
 ]
 
 
