@@ -294,7 +294,8 @@ def host_codes(w, kv):
     return wl.bf16_bits(w.kv_pool)
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """One process per GPU (torchrun env); `gloo` is for the CPU tests."""
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -302,22 +303,31 @@ def dist_setup():
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
 
-def max_over_ranks(x, ws):
+def max_over_ranks(x, ws, device="cuda"):
+    """Slowest rank's time: every timed number is the max over ranks."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_gbs(bytes_per_rank, t_step_max, ws):
+    """Whole-job KV GB/s: every replica reads its own bytes in the slowest time."""
+    return ws * bytes_per_rank / t_step_max / 1e9
 
 
 def barrier(ws):
@@ -358,7 +368,7 @@ def main():
     barrier(ws)
     t_step = max_over_ranks(statistics.median(total), ws)
     t_partial = max_over_ranks(statistics.median(partial), ws)
-    value = ws * w.kv_bytes / t_step / 1e9
+    value = job_gbs(w.kv_bytes, t_step, ws)
 
     e2e_t, h2d, d2h = run_e2e(w, kv, max(5, args.steps // 2), args.warmup)
     e2e_t = max_over_ranks(e2e_t, ws)
