@@ -9,8 +9,12 @@
 //    each writing a partial result (normalised O and its log-sum-exp) that a
 //    second kernel merges.
 //
-// One CTA = (query-row group g of up to 64 rows, split s, request b).  The
-// rows of a group are (q, h) pairs in [q_len][H] order.
+// Work unit = (query-row group g of up to 64 rows, split s, request b); the
+// rows of a group are (q, h) pairs in [q_len][H] order.  The grid is one-
+// dimensional: one CTA per unit, except that units can be cut into 2 or 4
+// contiguous runs of the split's tiles, one CTA each, launched as a cluster
+// that merges its results on chip (merge_pieces) - all units when they fill at
+// most half of the GPU, or only those of a partly filled last wave.
 //
 // Tensor-core mapping (tokens as M): with at most 64 query rows per CTA,
 // using the rows as M would run the half-width M=64 UMMA shape and would need
