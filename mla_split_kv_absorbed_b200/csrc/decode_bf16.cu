@@ -5,8 +5,9 @@
 // "更深的 MLA 流水线" (keep more KV reads in flight) and "更快的 split-KV 归约"
 // (per-CTA partial results merged by a second kernel).
 //
-// Same mapping as the FP8 kernel (tokens as UMMA M = 128, up to 64 query rows
-// as N, O^T accumulated in TMEM in four 128-dim blocks), with bf16 operands:
+// Tensor-core mapping as in the FP8 kernel (tokens as UMMA M = 128, up to 64
+// query rows as N, O^T accumulated in TMEM in four 128-dim blocks), with bf16
+// operands.  One CTA per (64-row query group, split, request), a 3-D grid:
 //   S^T[t][n] = K[t][:] . Q[n][:]        A = K chunk (K-major SW128), B = Q
 //   O^T[d][n] += V^T[d][t] . P[t][n]     A = V pair (MN-major SW128), B = P (bf16)
 // The query is exact in bf16, so no operand split is needed.
@@ -22,9 +23,11 @@
 // every KV byte once, and each slot is held only from its load until its
 // MMAs complete, which keeps up to 128 KiB of loads in flight.
 //
-// Warp roles and the softmax / rescale / epilogue logic are those of the FP8
-// kernel: producer (warp 0), warp-uniform MMA issuer (warp 1), two softmax
-// warpgroups (warps 4-11, 32 columns each), rescale + epilogue (warps 12-15).
+// Warp roles (512 threads): producer (warp 0), warp-uniform MMA issuer
+// (warp 1), two softmax warpgroups (warps 4-11, 32 query columns each, thread
+// = token row), O^T rescale between tiles and epilogue (warps 12-15, thread =
+// latent dim).  The online softmax (log2 domain, lazy running max moving only
+// when exceeded by more than 1) and the bounded waits follow the FP8 kernel.
 #include <cstdint>
 #include <cuda_bf16.h>
 
