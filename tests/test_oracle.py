@@ -169,6 +169,28 @@ def test_identical_keys_give_mean_and_log_length(oracle_lib):
         assert lse[h] == pytest.approx(s + math.log(150), rel=1e-12)
 
 
+def test_common_rope_key_shifts_lse_only(oracle_lib):
+    # When every token has the same RoPE key r, changing the RoPE query by d
+    # moves every score by softmax_scale * (d . r): the weights, and so O, do
+    # not change, and the LSE moves by exactly that amount.
+    rng = np.random.default_rng(5)
+    c = _case(rng, 1, 1, 2, [300], fp8=False)
+    r = c["kv_pages"][c["block_table"][0, 0], 0, 512:].copy()
+    c["kv_pages"][:, :, 512:] = r[None, None, :]
+    o, lse = _oracle_decode(oracle_lib, c)
+    c2 = dict(c)
+    qr2 = c["q_rope"].copy()
+    qr2[0, 0, :, 3] = np.float32(0.75).view(np.uint32) >> 16       # exact in bf16
+    qr2[0, 0, :, 40] = np.float32(-2.5).view(np.uint32) >> 16
+    c2["q_rope"] = qr2
+    o2, lse2 = _oracle_decode(oracle_lib, c2)
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-13)
+    rv = npr.bf16_bits_to_f64(r)
+    for h in range(2):
+        d = npr.bf16_bits_to_f64(qr2[0, 0, h]) - npr.bf16_bits_to_f64(c["q_rope"][0, 0, h])
+        assert lse2[h] - lse[h] == pytest.approx(c["softmax_scale"] * float(d @ rv), rel=1e-10, abs=1e-12)
+
+
 def test_zero_query_gives_mean_of_values(oracle_lib):
     rng = np.random.default_rng(3)
     c = _case(rng, 1, 1, 1, [97], fp8=True)
