@@ -171,6 +171,20 @@ MLA_API int mla_decode_noalloc(const uint16_t* q_nope, const uint16_t* q_rope,
 MLA_API int mla_choose_splits(const int32_t* seq_lens_host, int B, int q_len, int H,
                       int num_sms, int max_splits, int32_t* out_host);
 
+/* Host helper, no GPU needed: how mla_decode_partial lays out its CTAs for
+ * a problem shape on num_sms SMs.  Units are (64-row query group, split,
+ * request) triples.  FP8: when the units fill at most half of the SMs, every
+ * split is cut into 2 or 4 contiguous runs of tiles, one CTA each, launched as
+ * a cluster that merges on chip; when they fill several waves and the last
+ * wave is at most half full, only that wave's units are cut in two.  bf16: one
+ * CTA per unit.  The partials are the same either way (rounding aside).
+ * out4 (HOST, 4 int32) = {CTAs launched, pieces per cut unit, index of the
+ * first cut unit, idle CTAs placed before the cut units so that clusters
+ * align}.  Returns MLA_ERR_INVALID_ARG for non-positive sizes or an unknown
+ * kv_dtype. */
+MLA_API int mla_partial_grid(int B, int q_len, int H, int max_splits, int kv_dtype, int num_sms,
+                             int32_t* out4);
+
 /* ---------------------------------------------------------------------------
  * mla_debug_inject_stall: a test hook for the failure path; the pages have no
  * counterpart.  While enabled (enable != 0), every FP8 mla_decode_partial

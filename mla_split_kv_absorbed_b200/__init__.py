@@ -71,6 +71,8 @@ def _load_lib():
     lib.mla_choose_splits.restype = i32
     lib.mla_status_string.argtypes = [i32]
     lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_partial_grid.argtypes = [i32, i32, i32, i32, i32, i32, P]
+    lib.mla_partial_grid.restype = i32
     lib.mla_debug_inject_stall.argtypes = [i32]
     lib.mla_debug_inject_stall.restype = i32
     return lib
@@ -183,6 +185,15 @@ def mla_choose_splits(seq_lens_host, q_len: int, H: int, num_sms: int, max_split
 
 def mla_status_string(status: int) -> str:
     return status_string(status)
+
+
+def mla_partial_grid(B: int, q_len: int, H: int, max_splits: int, kv_dtype: int, num_sms: int):
+    """CTA layout mla_decode_partial uses: (ctas, pieces per cut unit, first
+    cut unit, idle CTAs before the cut units)."""
+    out = (ctypes.c_int32 * 4)()
+    _check("mla_partial_grid", _lib.mla_partial_grid(B, q_len, H, max_splits, kv_dtype, num_sms,
+                                                     ctypes.cast(out, ctypes.c_void_p)))
+    return tuple(int(v) for v in out)
 
 
 def mla_debug_inject_stall(enable: bool) -> bool:

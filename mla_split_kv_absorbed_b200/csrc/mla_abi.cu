@@ -77,6 +77,36 @@ int make_kv_map(CUtensorMap* map, const void* kv_pages, int kv_dtype, int64_t nu
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+// FP8 partial-kernel grid over units (64-row query group, split, request).
+// When the units fill at most half of the SMs, every split is cut into 2 or 4
+// runs of tiles, one CTA each, merged on chip by its cluster; when they fill
+// several waves and the last wave is at most half full, only the units of that
+// last wave are cut in two.  The partial per split is the same either way.
+// out = {CTAs, pieces, first cut unit, idle CTAs before the cut units}.
+void plan_grid(int B, int q_len, int H, int max_splits, int kv_dtype, int sms, int32_t* out) {
+  const long long groups = (q_len * H + 63) / 64;
+  const long long units = groups * max_splits * B;
+  int pieces = 1;
+  long long split_from = units;
+  if (kv_dtype == MLA_KV_FP8_E4M3 && sms > 0) {
+    if (units * 2 <= sms) {
+      while (pieces < 4 && units * pieces * 2 <= sms) pieces *= 2;
+      split_from = 0;
+    } else if (units > sms) {
+      const long long tail = units % sms;
+      if (tail > 0 && tail * 2 <= sms) {
+        pieces = 2;
+        split_from = units - tail;
+      }
+    }
+  }
+  const long long pad = pieces > 1 ? (pieces - split_from % pieces) % pieces : 0;
+  out[0] = (int32_t)(split_from + pad + (units - split_from) * pieces);
+  out[1] = pieces;
+  out[2] = (int32_t)split_from;
+  out[3] = (int32_t)pad;
+}
+
 }  // namespace
 
 extern "C" {
@@ -143,29 +173,13 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   a.qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
   a.kv_scale = kv_scale;
   a.inject_stall = g_inject_stall.load(std::memory_order_relaxed);
-  // FP8 path: when the (group, split, request) units fill at most half of the
-  // SMs, every split is cut into 2 or 4 runs of tiles, one CTA each, merged
-  // on chip by its cluster; when they fill several waves and the last wave is
-  // at most half full, only the units of that last wave are cut in two.  The
-  // partial per split is the same either way.
-  a.groups = (q_len * H + 63) / 64;
-  const long long units = (long long)a.groups * max_splits * B;
-  a.pieces = 1;
-  a.split_from = (int)units;
-  a.pad = 0;
-  if (kv_dtype == MLA_KV_FP8_E4M3) {
-    const int sms = num_sms_cached();
-    if (units * 2 <= sms) {
-      while (a.pieces < 4 && units * a.pieces * 2 <= sms) a.pieces *= 2;
-      a.split_from = 0;
-    } else if (units > sms) {
-      const long long tail = units % sms;
-      if (tail > 0 && tail * 2 <= sms) {
-        a.pieces = 2;
-        a.split_from = (int)(units - tail);
-      }
-    }
-    if (a.pieces > 1) a.pad = (a.pieces - a.split_from % a.pieces) % a.pieces;
+  {
+    int32_t plan[4];
+    plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms_cached(), plan);
+    a.groups = (q_len * H + 63) / 64;
+    a.pieces = plan[1];
+    a.split_from = plan[2];
+    a.pad = plan[3];
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, s)
@@ -218,6 +232,16 @@ const char* mla_status_string(int status) {
     case MLA_ERR_SCRATCH_LIMIT: return "MLA_ERR_SCRATCH_LIMIT";
     default: return "MLA_ERR_UNKNOWN";
   }
+}
+
+int mla_partial_grid(int B, int q_len, int H, int max_splits, int kv_dtype, int num_sms,
+                     int32_t* out4) {
+  if (out4 == nullptr || B < 1 || q_len < 1 || H < 1 || max_splits < 1 || num_sms < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (kv_dtype != MLA_KV_FP8_E4M3 && kv_dtype != MLA_KV_BF16) return MLA_ERR_INVALID_ARG;
+  plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms, out4);
+  if (kv_dtype == MLA_KV_BF16) out4[0] = ((q_len * H + 63) / 64) * max_splits * B;
+  return MLA_OK;
 }
 
 int mla_debug_inject_stall(int enable) {

@@ -104,3 +104,26 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(m, "_lib_handle", None)
     with pytest.raises(ImportError):
         m.load()
+
+
+def test_partial_grid_plan(lib):
+    # how mla_decode_partial lays out its CTAs (host logic, no GPU):
+    # (ctas, pieces per cut unit, first cut unit, idle CTAs before the cut units)
+    import mla_split_kv_absorbed_b200 as m
+    FP8, BF16 = m.MLA_KV_FP8_E4M3, m.MLA_KV_BF16
+    # batch 1, 64 heads, 64 splits: 64 units fill under half of 148 SMs -> every split cut in 2
+    assert m.mla_partial_grid(1, 1, 64, 64, FP8, 148) == (128, 2, 0, 0)
+    # a handful of units: cut in 4
+    assert m.mla_partial_grid(1, 1, 64, 4, FP8, 148) == (16, 4, 0, 0)
+    # batch 16, 32 splits: 512 units = 3 full waves + 68 -> the last 68 cut in 2
+    assert m.mla_partial_grid(16, 1, 64, 32, FP8, 148) == (444 + 136, 2, 444, 0)
+    # batch 4: 128 units, one wave more than half full -> no cut
+    assert m.mla_partial_grid(4, 1, 64, 32, FP8, 148) == (128, 1, 128, 0)
+    # q_len 4: 4 row groups x 64 splits x 8 -> last wave 124 > 74 -> no cut
+    assert m.mla_partial_grid(8, 4, 64, 64, FP8, 148) == (2048, 1, 2048, 0)
+    # odd first cut unit: one idle CTA keeps the 2-CTA clusters aligned
+    assert m.mla_partial_grid(1, 1, 64, 150, FP8, 147) == (147 + 1 + 6, 2, 147, 1)
+    # bf16 cache: one CTA per unit
+    assert m.mla_partial_grid(1, 1, 16, 4, BF16, 148)[0] == 4
+    with pytest.raises(m.MlaError):
+        m.mla_partial_grid(0, 1, 64, 4, FP8, 148)
