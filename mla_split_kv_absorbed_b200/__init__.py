@@ -12,6 +12,12 @@ Entry points (same names as the C ABI):
 * ``mla_decode_partial(...)`` — steps A2-A8, per-split partial O and LSE.
 * ``mla_combine(...)`` — step A9, log-sum-exp merge into bf16 O and fp32 LSE.
 * ``mla_partial_workspace_bytes``, ``mla_choose_splits``, ``mla_status_string``.
+* ``mla_partial_grid(...)`` — host helper: the partial kernel's CTA layout for a shape.
+* ``mla_debug_inject_stall(enable)`` — test hook for the bounded-wait failure path.
+
+``mla_decode_noalloc`` (partial + merge with in-library scratch) is reached
+through ``load()`` directly; its ctypes signature is in the GPU test that uses
+it.
 
 ``decode(...)`` chains partial + combine with a caller-provided or freshly
 allocated workspace.
@@ -32,7 +38,8 @@ MLA_KV_FP8_E4M3, MLA_KV_BF16 = 0, 1
 DEVERR_BAD_PAGE, DEVERR_BAD_SEQLEN, DEVERR_TIMEOUT, DEVERR_BAD_SPLITS, DEVERR_SMEM_ALIGN = 1, 2, 4, 8, 16
 
 EXPORTS = ("mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
-           "mla_combine", "mla_choose_splits", "mla_status_string")
+           "mla_combine", "mla_choose_splits", "mla_status_string", "mla_decode_noalloc",
+           "mla_partial_grid", "mla_debug_inject_stall")
 
 
 class MlaError(RuntimeError):
