@@ -16,6 +16,9 @@ Functions (each cites its passage in ``oracle.c``):
   (same article, bullet "更快的 split-KV 归约").
 * :func:`combine` — the log-sum-exp merge of the partials done by the second
   kernel (same bullet).
+* :func:`rope_f64`, :func:`rope_table`, :func:`append_kv` — the KV-append step
+  before the path: RoPE on the 64-wide key, saturating E4M3 and the paged
+  write ("Muse Spark Open" article, bullet "RoPE 与 KV 缓存写入融合").
 """
 from __future__ import annotations
 
@@ -62,6 +65,11 @@ def _load():
                                                  i32, i32, f32, P, i64, P, P]
         lib.oracle_combine.argtypes = [P, P, P, i32, i64, P, P]
         lib.oracle_num_threads.restype = i32
+        lib.oracle_rope_f64.argtypes = [P, i64, ctypes.c_double, P]
+        lib.oracle_rope_table.argtypes = [i64, ctypes.c_double, P]
+        lib.oracle_append_kv.argtypes = [P, P, P, i64, P, i32, P, i32, i32, f32, P, i64]
+        lib.oracle_append_kv.restype = i64
+        lib.oracle_set_num_threads.argtypes = [i32]
         _lib = lib
     return _lib
 
@@ -73,6 +81,11 @@ def _ptr(a: np.ndarray):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the following oracle calls (OpenMP); used to time it on one core."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def e4m3_value(code: int) -> float:
@@ -161,3 +174,37 @@ def combine(part_o: np.ndarray, part_lse: np.ndarray, n_splits: np.ndarray):
     lse = np.zeros(R, dtype=np.float64)
     lib.oracle_combine(_ptr(po), _ptr(pl), _ptr(ns), S, R, _ptr(o), _ptr(lse))
     return o, lse
+
+
+def rope_f64(x, pos: int, base: float = 10000.0) -> np.ndarray:
+    """RoPE of one 64-wide key in fp64 (pairs (2i, 2i+1), theta_i = base^(-2i/64))."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    assert x.shape == (D_ROPE,)
+    y = np.empty(D_ROPE, dtype=np.float64)
+    _load().oracle_rope_f64(_ptr(x), int(pos), float(base), _ptr(y))
+    return y
+
+
+def rope_table(max_pos: int, base: float = 10000.0) -> np.ndarray:
+    """fp32 [max_pos][32][2] (cos, sin) of pos * theta_i, each rounded once from fp64."""
+    t = np.empty((max_pos, D_ROPE // 2, 2), dtype=np.float32)
+    _load().oracle_rope_table(int(max_pos), float(base), _ptr(t))
+    return t
+
+
+def append_kv(c_kv_bits, k_rope_bits, cos_sin, block_table, seq_lens, n_new: int, inv_scale: float,
+              kv_pages: np.ndarray) -> int:
+    """Write n_new tokens per request into kv_pages (uint8 [num_pages][64][576], in
+    place).  c_kv_bits uint16 [B][n_new][512], k_rope_bits uint16 [B][n_new][64]
+    (bf16 bits).  Returns the number of tokens skipped as out of range."""
+    lib = _load()
+    c = np.ascontiguousarray(c_kv_bits, dtype=np.uint16)
+    r = np.ascontiguousarray(k_rope_bits, dtype=np.uint16)
+    cs = np.ascontiguousarray(cos_sin, dtype=np.float32)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    assert kv_pages.dtype == np.uint8 and kv_pages.flags["C_CONTIGUOUS"]
+    B = bt.shape[0]
+    return int(lib.oracle_append_kv(_ptr(c), _ptr(r), _ptr(cs), cs.shape[0], _ptr(bt), bt.shape[1],
+                                    _ptr(sl), B, int(n_new), float(np.float32(inv_scale)),
+                                    _ptr(kv_pages), kv_pages.shape[0]))

@@ -15,6 +15,9 @@
  *        a second kernel merges the partial results;
  *      bullet "原生 FP8 转换"          — KV/Q converted to FP8 with a
  *        saturating conversion: overflow clamps to +-448, never NaN.
+ *  - "Muse Spark Open" article (theainews.cc), section "内核优化：解码吞吐 3
+ *    倍", bullet "RoPE 与 KV 缓存写入融合" — RoPE applied in the kernel that
+ *    writes the decode KV cache (the KV-append step before the path).
  *  - The OCP 8-bit floating point specification (E4M3: bias 7, no infinity,
  *    S.1111.111 is NaN, largest finite 448) for the code <-> value map.
  *  - Absorbed MLA as a plain softmax(q k^T * scale) v over one 576-wide latent
@@ -306,7 +309,97 @@ void oracle_combine(const float* part_o, const float* part_lse, const int32_t* n
   }
 }
 
-/* Threads OpenMP will use (reported with CPU timings). */
+/* ------------------------------------------------------------------------ */
+/* KV append: RoPE on the 64-wide key, saturating E4M3, paged write          */
+/* ------------------------------------------------------------------------ */
+/*
+ * The step before the decode path: each new token's latent (512) and RoPE key
+ * (64) are written into the paged FP8 cache.  "Muse Spark Open" article
+ * (theainews.cc), section "内核优化：解码吞吐 3 倍", bullet "RoPE 与 KV 缓存写入
+ * 融合": the rotary embedding is applied in the same kernel that writes the
+ * decode KV cache; "SGLang & Miles ... Vera Rubin" article, bullet "原生 FP8
+ * 转换": KV is stored as saturating E4M3.  The pages print no RoPE formula;
+ * the reading here is the original rotary position embedding: consecutive
+ * dims (2i, 2i+1) of the 64-wide key rotated by the angle pos * theta_i with
+ * theta_i = base^(-2i/64).
+ */
+
+/* The rotation in fp64, straight from the definition (used by the pins). */
+void oracle_rope_f64(const double* x, int64_t pos, double base, double* y) {
+  for (int i = 0; i < D_ROPE / 2; ++i) {
+    const double theta = pow(base, -2.0 * i / (double)D_ROPE);
+    const double a = (double)pos * theta;
+    const double c = cos(a), s = sin(a);
+    y[2 * i] = x[2 * i] * c - x[2 * i + 1] * s;
+    y[2 * i + 1] = x[2 * i] * s + x[2 * i + 1] * c;
+  }
+}
+
+/* cos_sin[pos][i] = (fl32(cos(pos theta_i)), fl32(sin(pos theta_i))) for
+ * pos < max_pos, i < 32: the angle and its cosine and sine in fp64, each
+ * rounded once to fp32.  This is the cache of angles a serving engine keeps. */
+void oracle_rope_table(int64_t max_pos, double base, float* cos_sin) {
+  for (int64_t pos = 0; pos < max_pos; ++pos)
+    for (int i = 0; i < D_ROPE / 2; ++i) {
+      const double theta = pow(base, -2.0 * i / (double)D_ROPE);
+      const double a = (double)pos * theta;
+      cos_sin[(pos * (D_ROPE / 2) + i) * 2] = (float)cos(a);
+      cos_sin[(pos * (D_ROPE / 2) + i) * 2 + 1] = (float)sin(a);
+    }
+}
+
+/* Append n_new tokens per request.  Token j of request b has position
+ * pos = seq_lens[b] - n_new + j (seq_lens counts the new tokens) and goes to
+ * row pos % 64 of page block_table[b][pos / 64]:
+ *   latent dim d:   code = E4M3(fl32(x_d * inv_scale))
+ *   RoPE pair i:    with (c, s) = cos_sin[pos][i] and x0, x1 the pair's bf16
+ *                   values, in fp32 (each operation rounded, no fused
+ *                   multiply-add):  y0 = x0 c - x1 s,  y1 = x0 s + x1 c;
+ *                   codes E4M3(fl32(y * inv_scale)).
+ * Returns the number of tokens skipped because their position, page index or
+ * page id was out of range (those tokens are not written). */
+int64_t oracle_append_kv(const uint16_t* c_kv, const uint16_t* k_rope, const float* cos_sin,
+                         int64_t max_pos, const int32_t* block_table, int max_pages,
+                         const int32_t* seq_lens, int B, int n_new, float inv_scale,
+                         uint8_t* kv_pages, int64_t num_pages) {
+  init_tables();
+  int64_t skipped = 0;
+  for (int b = 0; b < B; ++b)
+    for (int j = 0; j < n_new; ++j) {
+      const int64_t pos = (int64_t)seq_lens[b] - n_new + j;
+      if (pos < 0 || pos >= max_pos || pos / PAGE >= max_pages) { ++skipped; continue; }
+      const int64_t page = block_table[(int64_t)b * max_pages + pos / PAGE];
+      if (page < 0 || page >= num_pages) { ++skipped; continue; }
+      uint8_t* row = kv_pages + (page * PAGE + pos % PAGE) * D_ROW;
+      const uint16_t* xc = c_kv + ((int64_t)b * n_new + j) * D_LATENT;
+      const uint16_t* xr = k_rope + ((int64_t)b * n_new + j) * D_ROPE;
+      for (int d = 0; d < D_LATENT; ++d) {
+        volatile float p = bf16_to_f32(xc[d]) * inv_scale;
+        row[d] = oracle_e4m3_encode(p);
+      }
+      for (int i = 0; i < D_ROPE / 2; ++i) {
+        const float c = cos_sin[(pos * (D_ROPE / 2) + i) * 2];
+        const float s = cos_sin[(pos * (D_ROPE / 2) + i) * 2 + 1];
+        const float x0 = bf16_to_f32(xr[2 * i]), x1 = bf16_to_f32(xr[2 * i + 1]);
+        volatile float x0c = x0 * c, x1s = x1 * s, x0s = x0 * s, x1c = x1 * c;
+        volatile float y0 = x0c - x1s, y1 = x0s + x1c;
+        volatile float p0 = y0 * inv_scale, p1 = y1 * inv_scale;
+        row[D_LATENT + 2 * i] = oracle_e4m3_encode(p0);
+        row[D_LATENT + 2 * i + 1] = oracle_e4m3_encode(p1);
+      }
+    }
+  return skipped;
+}
+
+/* Threads OpenMP will use (reported with CPU timings); the setter lets a
+ * timing run the same code on one core. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -307,3 +307,133 @@ def test_combine_closed_forms(oracle_lib):
     assert np.all(o[1] == 0) and lse[1] == -np.inf
     np.testing.assert_allclose(o[2], po[2, 0].astype(np.float64), rtol=0, atol=0)
     assert lse[2] == pytest.approx(2.0)
+
+
+# --------------------------------------------------------------------------- KV append
+# The step before the path: RoPE on the 64-wide key, saturating E4M3, paged
+# write ("Muse Spark Open" article, section "内核优化：解码吞吐 3 倍", bullet
+# "RoPE 与 KV 缓存写入融合"; "SGLang & Miles ... Vera Rubin" article, bullet
+# "原生 FP8 转换").  Reading: the original rotary embedding, pairs (2i, 2i+1),
+# theta_i = 10000^(-2i/64).
+
+def test_rope_position_zero_is_identity_and_norm_is_kept(oracle_lib):
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal(64)
+    assert np.array_equal(oracle_lib.rope_f64(x, 0), x)
+    for pos in (1, 7, 4095, 131071, 262143):
+        y = oracle_lib.rope_f64(x, pos)
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-12
+        # each pair keeps its own length (a rotation acts within the pair)
+        assert np.allclose(np.hypot(y[0::2], y[1::2]), np.hypot(x[0::2], x[1::2]), rtol=0, atol=1e-12)
+
+
+def test_rope_closed_form_pairs(oracle_lib):
+    # pair 0 has theta = 1: a rotation by pos radians; pair 16 has theta = 10000^-0.5 = 0.01
+    x = np.zeros(64)
+    x[0], x[1] = 1.0, 0.0
+    x[32], x[33] = 0.0, 2.0
+    y = oracle_lib.rope_f64(x, 3)
+    assert abs(y[0] - math.cos(3.0)) < 1e-15 and abs(y[1] - math.sin(3.0)) < 1e-15
+    assert abs(y[32] - (-2.0 * math.sin(0.03))) < 1e-15 and abs(y[33] - 2.0 * math.cos(0.03)) < 1e-15
+
+
+def test_rope_composes_and_relative_positions(oracle_lib):
+    # R(a) R(b) = R(a + b), and <R(m) q, R(n) k> depends only on m - n
+    rng = np.random.default_rng(12)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    a, b = 37, 1000
+    # rotating by a then by b: apply the pairwise rotation of b to R(a) x
+    ra = oracle_lib.rope_f64(q, a)
+    rab = oracle_lib.rope_f64(ra, b)
+    assert np.allclose(rab, oracle_lib.rope_f64(q, a + b), rtol=0, atol=1e-11)
+    d1 = oracle_lib.rope_f64(q, 500) @ oracle_lib.rope_f64(k, 480)
+    d2 = oracle_lib.rope_f64(q, 20) @ oracle_lib.rope_f64(k, 0)
+    assert abs(d1 - d2) < 1e-11
+
+
+def test_rope_table_is_the_rounded_angles(oracle_lib):
+    t = oracle_lib.rope_table(300)
+    pos = np.arange(300)[:, None]
+    theta = 10000.0 ** (-2.0 * np.arange(32) / 64.0)
+    ang = pos * theta[None, :]
+    assert np.array_equal(t[..., 0], np.cos(ang).astype(np.float32))
+    assert np.array_equal(t[..., 1], np.sin(ang).astype(np.float32))
+    assert np.all(t[0, :, 0] == 1.0) and np.all(t[0, :, 1] == 0.0)
+
+
+def _append_case(seed=13, B=3, n_new=2, lens=(5, 64, 130), spare=3):
+    rng = np.random.default_rng(seed)
+    pages = [(L + 63) // 64 for L in lens]
+    num_pages = sum(pages) + spare
+    perm = rng.permutation(num_pages).astype(np.int32)
+    bt = np.full((B, max(pages)), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(pages):
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    c = rng.standard_normal((B, n_new, 512)).astype(np.float32)
+    r = (3.0 * rng.standard_normal((B, n_new, 64))).astype(np.float32)
+    bits = lambda a: (a.view(np.uint32) >> 16).astype(np.uint16)  # truncate to bf16 bits
+    return bits(c), bits(r), bt, np.array(lens, dtype=np.int32), num_pages
+
+
+def test_append_places_rows_and_quantises_the_latent_like_the_prep_step(oracle_lib):
+    c, r, bt, sl, num_pages = _append_case()
+    B, n_new = c.shape[:2]
+    inv = float(np.float32(448.0 / 8.0))
+    table = oracle_lib.rope_table(256)
+    kv = np.full((num_pages, 64, 576), 0xAA, dtype=np.uint8)
+    assert oracle_lib.append_kv(c, r, table, bt, sl, n_new, inv, kv) == 0
+    written = np.zeros((num_pages, 64), dtype=bool)
+    for b in range(B):
+        for j in range(n_new):
+            pos = sl[b] - n_new + j
+            page, row = bt[b, pos // 64], pos % 64
+            written[page, row] = True
+            # latent: the same codes as the (independently pinned) quantiser
+            assert np.array_equal(kv[page, row, :512], oracle_lib.quantize(c[b, j], inv))
+    # nothing else was touched
+    assert np.all(kv[~written] == 0xAA)
+
+
+def test_append_rope_codes_follow_the_fp64_rotation(oracle_lib):
+    # the fp32 rotation rounds a few times; its codes equal the E4M3 rounding of
+    # the exact fp64 rotation except where y * inv_scale lies within a few fp32
+    # ulps of a rounding boundary, and then they are neighbours
+    rng = np.random.default_rng(14)
+    B, n_new, L = 1, 64, 100000
+    c = np.zeros((B, n_new, 512), dtype=np.uint16)
+    rf = (4.0 * rng.standard_normal((B, n_new, 64))).astype(np.float32)
+    r = (rf.view(np.uint32) >> 16).astype(np.uint16)
+    bt = np.arange((L + 63) // 64, dtype=np.int32)[None, :]
+    kv = np.zeros((bt.shape[1], 64, 576), dtype=np.uint8)
+    inv = float(np.float32(448.0 / 16.0))
+    table = oracle_lib.rope_table(L)
+    assert oracle_lib.append_kv(c, r, table, bt, np.array([L], np.int32), n_new, inv, kv) == 0
+    vals = lambda codes: np.array([oracle_lib.e4m3_value(int(v)) for v in codes])
+    diffs = 0
+    for j in range(n_new):
+        pos = L - n_new + j
+        x = (r[0, j].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        y = oracle_lib.rope_f64(x, pos) * inv
+        got = kv[pos // 64, pos % 64, 512:]
+        want = npr.e4m3_round(y.astype(np.float32))
+        mism = got != want
+        diffs += int(mism.sum())
+        if mism.any():
+            # neighbouring codes only, and only near a rounding boundary
+            assert np.all(np.abs(vals(got[mism]) - vals(want[mism])) <=
+                          2 * np.abs(vals(want[mism])) * 2.0 ** -3 + 2.0 ** -9)
+    assert diffs <= n_new * 64 // 100
+
+
+def test_append_skips_out_of_range_tokens(oracle_lib):
+    c, r, bt, sl, num_pages = _append_case()
+    kv = np.zeros((num_pages, 64, 576), dtype=np.uint8)
+    table = oracle_lib.rope_table(100)  # request 2 ends at position 129: beyond the table
+    skipped = oracle_lib.append_kv(c, r, table, bt, sl, 2, 1.0, kv)
+    assert skipped == 2
+    bt2 = bt.copy()
+    bt2[0, 0] = num_pages + 5  # page id outside the pool
+    kv2 = np.zeros_like(kv)
+    assert oracle_lib.append_kv(c, r, oracle_lib.rope_table(256), bt2, sl, 2, 1.0, kv2) == 2
