@@ -7,10 +7,14 @@ produced once per run by mla_quantize_fp8 (step A1), which is timed on its
 own and reported under "quantize".
 
 Default workload: batch 1, q_len 1, 64 heads, 128K context, FP8 E4M3 paged
-KV (page 64, shuffled block table), 64-way split.  The batch-16 workload (same
-shape, 32-way split) is measured in the same run and reported under
-"batch16".  L2 is flushed (a 256 MiB write) before every timed step, outside
-the timed events, so the 75.5 MB batch-1 cache is read from HBM.
+KV (page 64, shuffled block table), 64-way split.  The other four workloads
+are measured in the same run, each under its own key: "tiny" (batch 1, 16
+heads, 1024 tokens, bf16), "batch16" (batch 16 at 128K, FP8, 32-way split),
+"ragged_b32_bf16" (batch 32, 128 heads, ragged lengths, bf16) and
+"verify_q4_256k" (batch 8, q_len 4 causal, 256K, FP8; tensor-bound, so its
+roofline is against the bf16 tensor peak).  L2 is flushed (a 256 MiB write)
+before every timed step, outside the timed events, so the 75.5 MB batch-1
+cache is read from HBM.
 
 value = KV bytes read per step (sum_b L_b * 576) over all ranks / step time,
 in GB/s; ms_per_step is the device time of one step (max over ranks).
@@ -37,15 +41,17 @@ sys.path.insert(0, ROOT)
 METRIC = "MLA decode µs/step and KV-read HBM GB/s (% of peak) at 128K ctx, batch 1/16"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def load_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, "measured" | "fallback")."""
     try:
         with open(PEAKS_FILE) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 class ClockSampler:
@@ -261,28 +267,71 @@ def run_e2e(w, kv, steps, warmup):
     return statistics.median(times), h2d, d2h
 
 
-def cpu_baseline(w, kv_codes_host, budget_s=12.0):
-    """The oracle, as it stands, on a bounded sample: whole query rows of the
-    workload (all tokens of the row), as many as fit in about budget_s; the
-    projected full-step time gives the same GB/s metric."""
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _oracle_rows_rate(w, codes, budget_s, threads):
+    """Oracle decode of whole query rows on `threads` cores for about budget_s:
+    (rows done, seconds, projected seconds for a full step)."""
     import numpy as np
     import oracle
     from mla_split_kv_absorbed_b200 import workloads as wl
     qn, qr = wl.bf16_bits(w.q_nope), wl.bf16_bits(w.q_rope)
     bt, sl = w.block_table.cpu().numpy(), w.seq_lens.cpu().numpy()
     R = w.B * w.q_len * w.H
-    threads = oracle.num_threads()
+    oracle.set_num_threads(threads)
     rows_done, t_used, batch = 0, 0.0, threads
     while t_used < budget_s and rows_done < R:
         rows = np.arange(rows_done, min(R, rows_done + batch), dtype=np.int64)
         t0 = time.perf_counter()
-        oracle.decode_rows(qn, qr, kv_codes_host, w.kv_scale, bt, sl, w.q_len, w.H, w.softmax_scale, rows)
+        oracle.decode_rows(qn, qr, codes, w.kv_scale, bt, sl, w.q_len, w.H, w.softmax_scale, rows)
         t_used += time.perf_counter() - t0
         rows_done += rows.size
-    t_step = t_used * R / rows_done
+    return rows_done, t_used, t_used * R / rows_done
+
+
+def cpu_baseline(w, kv_codes_host, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample: whole query rows of the
+    workload (all tokens of the row), as many as fit in about budget_s on all
+    host cores; the projected full-step time gives the same GB/s metric.  Also
+    on one core for the tiny and batch-1 workloads, and the quantiser."""
+    import numpy as np
+    import oracle
+    from mla_split_kv_absorbed_b200 import workloads as wl
+    all_threads = os.cpu_count() or 1
+    oracle.set_num_threads(all_threads)
+    threads = oracle.num_threads()
+    R = w.B * w.q_len * w.H
+    rows_done, t_used, t_step = _oracle_rows_rate(w, kv_codes_host, budget_s, threads)
+    one_core = {}
+    tiny = wl.make("tiny")
+    r1, t1, ts1 = _oracle_rows_rate(tiny, host_codes(tiny, None), 2.0, 1)
+    one_core["tiny"] = {"value": tiny.kv_bytes / ts1 / 1e9, "unit": "GB/s", "us_per_step": ts1 * 1e6,
+                        "sample": f"{r1} of {tiny.B * tiny.H} rows, {t1:.2f} s"}
+    r2, t2, ts2 = _oracle_rows_rate(w, kv_codes_host, 4.0, 1)
+    one_core[w.spec.name] = {"value": w.kv_bytes / ts2 / 1e9, "unit": "GB/s", "s_per_step": ts2,
+                             "sample": f"{r2} of {R} rows, {t2:.2f} s"}
+    oracle.set_num_threads(all_threads)
+    # quantiser: step A1 over the first 16M values of the pool, GB/s of 3 B/element
+    x = wl.bf16_bits(w.kv_pool).reshape(-1)[: 1 << 24]
+    t0 = time.perf_counter()
+    oracle.quantize(x, w.inv_scale)
+    tq = time.perf_counter() - t0
     return {"value": w.kv_bytes / t_step / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{rows_done} of {R} query rows (all {int(sl.max())} tokens each), "
-                      f"{t_used:.1f} s, projected to a full step ({t_step:.1f} s)"}
+            "cpu_model": cpu_model(),
+            "sample": f"{rows_done} of {R} query rows (all {int(w.seq_lens.max())} tokens each), "
+                      f"{t_used:.1f} s, projected to a full step ({t_step:.1f} s)",
+            "one_core": one_core,
+            "quantize": {"value": 3.0 * x.size / tq / 1e9, "unit": "GB/s", "cores": threads,
+                         "elements": int(x.size), "s": tq}}
 
 
 def host_codes(w, kv):
@@ -292,6 +341,52 @@ def host_codes(w, kv):
     if w.spec.kv_dtype == "fp8":
         return oracle.quantize(wl.bf16_bits(w.kv_pool), w.inv_scale)
     return wl.bf16_bits(w.kv_pool)
+
+
+def pct(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, int(q * len(xs)))]
+
+
+def flops_per_step(w):
+    """Algorithmic flops of one step: 2 (576 + 512) per visible token per query row."""
+    sl = w.seq_lens.cpu().tolist()
+    tok_rows = sum(w.H * (L - w.q_len + 1 + q) for L in sl for q in range(w.q_len))
+    return 2 * (576 + 512) * tok_rows
+
+
+def measure(name, steps, warmup, peak_hbm, peak_tflops, ws):
+    """One workload: step and partial-kernel times (median, p10, p90) and the
+    partial kernel's roofline (HBM, or tensor for the q_len-4 verify)."""
+    import torch
+    w, kv = setup_workload(name, "cuda")
+    if w.spec.splits == "by_length":
+        # the library's own split rule gives the same counts as the workload
+        import mla_split_kv_absorbed_b200 as m
+        chosen = m.mla_choose_splits(w.seq_lens.cpu(), 148, 64)
+        assert torch.equal(chosen, w.num_splits.cpu()), "mla_choose_splits disagrees with the workload"
+    tot, par = run_steps(w, kv, steps, warmup)
+    t = max_over_ranks(statistics.median(tot), ws)
+    tp = max_over_ranks(statistics.median(par), ws)
+    res = {"workload": name, "B": w.B, "q_len": w.q_len, "H": w.H, "kv": w.spec.kv_dtype,
+           "num_splits": w.max_splits, "kv_bytes_per_step": w.kv_bytes, "steps": steps,
+           "us_per_step": t * 1e6, "us_p10": pct(tot, 0.1) * 1e6, "us_p90": pct(tot, 0.9) * 1e6,
+           "kv_gbs": w.kv_bytes / t / 1e9, "frac_of_peak": w.kv_bytes / t / 1e9 / peak_hbm,
+           "partial_us": tp * 1e6, "partial_p10": pct(par, 0.1) * 1e6,
+           "partial_p90": pct(par, 0.9) * 1e6, "partial_gbs": w.kv_bytes / tp / 1e9}
+    kernel = "decode_fp8_kernel" if w.spec.kv_dtype == "fp8" else "decode_bf16_kernel"
+    if w.q_len > 1:
+        fl = flops_per_step(w)
+        res["roofline"] = {"bound": "tensor", "achieved": fl / tp / 1e12, "peak": peak_tflops,
+                           "unit": "TFLOP/s", "frac": fl / tp / 1e12 / peak_tflops,
+                           "algorithmic_flops": fl, "kernel": kernel}
+    else:
+        res["roofline"] = {"bound": "hbm", "achieved": w.kv_bytes / tp / 1e9, "peak": peak_hbm,
+                           "unit": "GB/s", "frac": w.kv_bytes / tp / 1e9 / peak_hbm,
+                           "traffic": recorded_traffic(kernel, name), "kernel": kernel}
+    del kv, w
+    torch.cuda.empty_cache()
+    return res
 
 
 def dist_setup(backend="nccl"):
@@ -336,6 +431,14 @@ def barrier(ws):
         dist.barrier()
 
 
+EXTRA_WORKLOADS = [
+    ("tiny", "tiny"),                              # B1 H16 L1024 bf16, 4 splits
+    ("batch16", "b16_128k_fp8"),                   # B16 H64 L128K FP8, 32 splits
+    ("ragged_b32_bf16", "b32_ragged_bf16"),        # B32 H128 ragged bf16, splits by length
+    ("verify_q4_256k", "verify_q4_256k_fp8"),      # B8 q_len 4 H64 L256K FP8, 64 splits
+]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,17 +446,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="b1_128k_fp8")
-    ap.add_argument("--no-batch16", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time only the main workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
 
     if args.impl == "reference":
         return reference_arm(args)
 
     import torch
-    import mla_split_kv_absorbed_b200 as m
     ws, rank, local = dist_setup()
-    peak, peak_kind = load_peaks()
+    peak, peak_tf, peak_kind = load_peaks()
 
     w, kv = setup_workload(args.workload, "cuda")
     quant = time_quantize(w, kv) if w.spec.kv_dtype == "fp8" else None
@@ -374,17 +478,12 @@ def main():
     e2e_t = max_over_ranks(e2e_t, ws)
 
     extra = {}
-    if not args.no_batch16 and args.workload == "b1_128k_fp8":
-        w16, kv16 = setup_workload("b16_128k_fp8", "cuda")
-        tot16, par16 = run_steps(w16, kv16, max(5, args.steps // 2), args.warmup)
-        t16 = max_over_ranks(statistics.median(tot16), ws)
-        p16 = max_over_ranks(statistics.median(par16), ws)
-        extra["batch16"] = {"workload": "b16_128k_fp8", "us_per_step": t16 * 1e6,
-                            "kv_gbs": w16.kv_bytes / t16 / 1e9,
-                            "frac_of_peak": w16.kv_bytes / t16 / 1e9 / peak,
-                            "partial_us": p16 * 1e6, "partial_gbs": w16.kv_bytes / p16 / 1e9}
-        del kv16, w16
-        torch.cuda.empty_cache()
+    if not args.no_extra:
+        with ClockSampler(local) as clk_x:
+            for key, name in EXTRA_WORKLOADS:
+                if name != args.workload:
+                    extra[key] = measure(name, args.steps, args.warmup, peak, peak_tf, ws)
+        extra["clocks_extra"] = clk_x.summary()
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -401,6 +500,8 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": t_step * 1e3,
         "us_per_step": t_step * 1e6,
+        "us_p10": pct(total, 0.1) * 1e6,
+        "us_p90": pct(total, 0.9) * 1e6,
         "frac_of_peak": w.kv_bytes / t_step / 1e9 / peak,
         "higher_is_better": True,
         "scaling": "weak",
@@ -416,7 +517,9 @@ def main():
                      "frac": achieved / peak,
                      "traffic": recorded_traffic(kernel_name, args.workload),
                      "algorithmic_bytes": w.kv_bytes,
-                     "kernel": kernel_name, "kernel_us": t_partial * 1e6, "peak_kind": peak_kind},
+                     "kernel": kernel_name, "kernel_us": t_partial * 1e6,
+                     "kernel_p10": pct(partial, 0.1) * 1e6, "kernel_p90": pct(partial, 0.9) * 1e6,
+                     "peak_kind": peak_kind},
         "e2e": {"value": ws * w.kv_bytes / e2e_t / 1e9, "unit": "GB/s", "us_per_step": e2e_t * 1e6,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,

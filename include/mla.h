@@ -32,8 +32,10 @@
  *   - Arrays are dense, C order, as laid out below.  Device pointers must be
  *     16-byte aligned (mla_quantize_fp8 also accepts unaligned pointers).
  *   - Return 0 (MLA_OK) or one of the MLA_ERR_* codes; nothing is launched when
- *     an argument is rejected.  No exceptions, no logging, no global state
- *     other than a per-process cache of the device's SM count.
+ *     an argument is rejected.  No exceptions, no logging.  The only global
+ *     state is per device and thread-safe: each device's SM count, looked up
+ *     on first use, and the kernels' shared-memory opt-in, set on every launch.
+ *     Calls may target any device the caller makes current.
  */
 #ifndef MLA_B200_H
 #define MLA_B200_H
@@ -56,7 +58,7 @@ enum {
   MLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, out of range */
   MLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. H*q_len not a multiple of 16) */
   MLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed */
-  MLA_ERR_DEVICE = 4,       /* reserved for callers that fold dev_error into a status */
+  MLA_ERR_DEVICE = 4,       /* the GPU set dev_error (mla_device_error_status) */
   MLA_ERR_SCRATCH_LIMIT = 5 /* mla_decode_noalloc: problem larger than its fixed scratch */
 };
 
@@ -86,8 +88,10 @@ enum {
 MLA_API int mla_quantize_fp8(const uint16_t* x_bf16, uint8_t* y_e4m3, int64_t n,
                      float inv_scale, void* stream);
 
-/* Bytes of the split workspace: part_o (B*q_len*H*max_splits*512 fp32)
- * followed by part_lse (B*q_len*H*max_splits fp32).  Returns 0 for invalid
+/* Bytes of the split workspace that holds the per-split partial results
+ * (article bullet "更快的 split-KV 归约": each CTA's partial result, merged
+ * by the second kernel): part_o (B*q_len*H*max_splits*512 fp32) followed by
+ * part_lse (B*q_len*H*max_splits fp32).  Returns 0 for invalid
  * sizes.  A caller may carve both arrays from one allocation of this size
  * (part_lse = part_o + B*q_len*H*max_splits*512). */
 MLA_API size_t mla_partial_workspace_bytes(int B, int q_len, int H, int max_splits);
@@ -111,7 +115,7 @@ MLA_API size_t mla_partial_workspace_bytes(int B, int q_len, int H, int max_spli
  *   part_lse[B][q_len][H][max_splits]      fp32  LSE_s (natural log of the
  *           scaled-score sum); an empty split gives O_s = 0, LSE_s = -inf.
  * softmax_scale multiplies q.k; kv_scale (FP8 only) multiplies every code.
- * Supported: H*q_len a multiple of 16, q_len in 1..4, H in 1..128,
+ * Supported: H*q_len a multiple of 16 and at most 512, q_len in 1..4,
  * max_splits in 1..256.  dev_error may be NULL.
  * ------------------------------------------------------------------------- */
 MLA_API int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope,
@@ -136,6 +140,30 @@ MLA_API int mla_combine(const float* part_o, const float* part_lse, const int32_
                 float* out_lse, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Sequence-sharded decode over several GPUs (the merge of "更快的 split-KV 归约"
+ * one level up): each rank holds a disjoint page range of every request, runs
+ * mla_decode_partial over it, folds its own splits into one partial per row
+ * with mla_combine_f32, the ranks exchange those (an all-gather of
+ * rows*513 fp32 per rank), and mla_merge_rank_partials merges them.
+ *
+ * mla_combine_f32: the merge of mla_combine with an fp32 output and the
+ * merged LSE: out_o [B][q_len][H][512] fp32, out_lse [B][q_len][H] fp32 (both
+ * required).  A row whose splits are all empty gives O = 0, LSE = -inf.
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_combine_f32(const float* part_o, const float* part_lse,
+                            const int32_t* num_splits, int max_splits, int B, int q_len, int H,
+                            float* out_o, float* out_lse, void* stream);
+
+/* mla_merge_rank_partials: rank_o [n_ranks][B][q_len][H][512] fp32 and
+ * rank_lse [n_ranks][B][q_len][H] fp32 (each rank's mla_combine_f32 output,
+ * stacked in rank order, as an all-gather lays them out) -> out_bf16
+ * [B][q_len][H][512] (nearest-even) and out_lse (nullable), by the same LSE
+ * merge over the ranks.  n_ranks in 1..256. */
+MLA_API int mla_merge_rank_partials(const float* rank_o, const float* rank_lse, int n_ranks,
+                                    int B, int q_len, int H, uint16_t* out_bf16, float* out_lse,
+                                    void* stream);
+
+/* ---------------------------------------------------------------------------
  * Allocation-free decode (steps A2-A9 in one call).  The pages have no
  * counterpart to this entry point; it exists for callers that cannot allocate
  * device memory (a plugin whose host owns the whole device memory pool and
@@ -150,7 +178,9 @@ MLA_API int mla_combine(const float* part_o, const float* part_lse, const int32_
  *     array (8192*513 fp32, about 16 MiB) until the process exits.
  *   - The first call on each device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress); make that first call before
- *     any stream capture.  Later calls reuse the address.
+ *     any stream capture.  Later calls reuse the address while the device's
+ *     CUDA context stays the same; after cudaDeviceReset (a new context) the
+ *     next call looks it up again, so make that call outside a capture too.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents.  Each call writes every entry it reads, so nothing needs to
  *     start at zero, but calls that overlap on the GPU (different streams,
@@ -165,11 +195,60 @@ MLA_API int mla_decode_noalloc(const uint16_t* q_nope, const uint16_t* q_rope,
                                int H, float softmax_scale, uint16_t* out_bf16, float* out_lse,
                                int32_t* dev_error, void* stream);
 
-/* Host helper (article bullet "64 路 split-KV"): per-request split counts that
- * keep about two waves of CTAs on num_sms SMs, at least 16 pages per split,
- * clamped to [1, max_splits].  seq_lens_host/out_host are HOST arrays of B. */
-MLA_API int mla_choose_splits(const int32_t* seq_lens_host, int B, int q_len, int H,
-                      int num_sms, int max_splits, int32_t* out_host);
+/* ---------------------------------------------------------------------------
+ * KV append, the step before the decode path ("Muse Spark Open" article,
+ * section "内核优化：解码吞吐 3 倍", bullet "RoPE 与 KV 缓存写入融合": RoPE is
+ * applied in the kernel that writes the decode KV cache; "SGLang & Miles ...
+ * Vera Rubin" article, bullet "原生 FP8 转换": saturating E4M3 storage).
+ *
+ * c_kv       [B][n_new][512] bf16   new tokens' compressed latent
+ * k_rope     [B][n_new][64]  bf16   new tokens' RoPE key, before rotation
+ * cos_sin    [max_pos][32][2] fp32  (cos, sin) of pos * theta_i, theta_i =
+ *            base^(-2i/64) (see mla_rope_cos_sin_table)
+ * block_table[B][max_pages_per_req], seq_lens [B] (lengths including the
+ *            n_new tokens, as for mla_decode_partial)
+ * kv_pages   [num_pages][64][576] E4M3 codes, written in place
+ * Token j of request b has position pos = seq_lens[b] - n_new + j and is
+ * written to row pos % 64 of page block_table[b][pos / 64]:
+ *   latent d:   E4M3_satfinite(fl32(x_d * inv_scale))
+ *   RoPE pair i (dims 2i, 2i+1), (c, s) = cos_sin[pos][i], fp32 with every
+ *   operation rounded to nearest and no fused multiply-add:
+ *     y0 = x0*c - x1*s,  y1 = x0*s + x1*c;  codes E4M3_satfinite(fl32(y*inv_scale)).
+ * A token whose position is outside [0, max_pos) or beyond the block table
+ * sets MLA_DEVERR_BAD_SEQLEN, one whose page id is outside [0, num_pages) sets
+ * MLA_DEVERR_BAD_PAGE; such tokens are not written, the others are.
+ * c_kv and kv_pages must be 16-byte aligned, k_rope 4-byte, cos_sin 8-byte.
+ * n_new may be 0.  dev_error may be NULL.
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_append_kv_fp8(const uint16_t* c_kv, const uint16_t* k_rope, const float* cos_sin,
+                              int64_t max_pos, const int32_t* block_table,
+                              int max_pages_per_req, const int32_t* seq_lens, int B, int n_new,
+                              float inv_scale, uint8_t* kv_pages, int64_t num_pages,
+                              int32_t* dev_error, void* stream);
+
+/* Host helper for mla_append_kv_fp8: fills the HOST array cos_sin_host
+ * [max_pos][32][2] with (cos, sin) of pos * base^(-2i/64), each computed in
+ * double and rounded once to fp32 (the original rotary embedding; base is
+ * 10000 in the paper that introduced it).  base must be > 1. */
+MLA_API int mla_rope_cos_sin_table(float* cos_sin_host, int64_t max_pos, double base);
+
+/* Host helper (article bullet "64 路 split-KV": batch-1 decode needs enough
+ * splits to occupy the SMs; the pages fix no rule, so this is a reading):
+ * one split per 2048 tokens of each request,
+ *   out_host[b] = min(max_splits, max(1, ceil(seq_lens_host[b] / 2048))),
+ * which gives 64 splits for a 128K-token request.  The rule itself does not
+ * depend on num_sms: when the resulting grid underfills the GPU,
+ * mla_decode_partial cuts each split across a CTA cluster on its own (see
+ * mla_partial_grid).  num_sms (the target's SM count, > 0) is validated only.
+ * seq_lens_host and out_host are HOST arrays of B int32; every seq_len must
+ * be >= 1.  Returns MLA_ERR_INVALID_ARG for null pointers or sizes <= 0. */
+MLA_API int mla_choose_splits(const int32_t* seq_lens_host, int B, int num_sms, int max_splits,
+                              int32_t* out_host);
+
+/* Fold a device error word (read back from dev_error after the stream has
+ * synchronised) into a status: MLA_OK for 0, MLA_ERR_DEVICE otherwise (the
+ * MLA_DEVERR_* bits say what the GPU found). */
+MLA_API int mla_device_error_status(int32_t dev_error_word);
 
 /* Host helper, no GPU needed: how mla_decode_partial lays out its CTAs for
  * a problem shape on num_sms SMs.  Units are (64-row query group, split,

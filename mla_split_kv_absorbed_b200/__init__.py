@@ -12,6 +12,11 @@ Entry points (same names as the C ABI):
 * ``mla_decode_partial(...)`` — steps A2-A8, per-split partial O and LSE.
 * ``mla_combine(...)`` — step A9, log-sum-exp merge into bf16 O and fp32 LSE.
 * ``mla_partial_workspace_bytes``, ``mla_choose_splits``, ``mla_status_string``.
+* ``mla_append_kv_fp8(...)`` — the KV-append step before the path: RoPE on the
+  64-wide key, saturating E4M3 and the paged write in one kernel;
+  ``mla_rope_cos_sin_table(max_pos)`` builds its (cos, sin) table.
+* ``mla_device_error_status(word)`` / ``check_device_error(dev_error)`` — fold
+  the GPU's error word into MLA_ERR_DEVICE.
 * ``mla_partial_grid(...)`` — host helper: the partial kernel's CTA layout for a shape.
 * ``mla_debug_inject_stall(enable)`` — test hook for the bounded-wait failure path.
 
@@ -38,8 +43,10 @@ MLA_KV_FP8_E4M3, MLA_KV_BF16 = 0, 1
 DEVERR_BAD_PAGE, DEVERR_BAD_SEQLEN, DEVERR_TIMEOUT, DEVERR_BAD_SPLITS, DEVERR_SMEM_ALIGN = 1, 2, 4, 8, 16
 
 EXPORTS = ("mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
-           "mla_combine", "mla_choose_splits", "mla_status_string", "mla_decode_noalloc",
-           "mla_partial_grid", "mla_debug_inject_stall")
+           "mla_combine", "mla_choose_splits", "mla_device_error_status", "mla_status_string",
+           "mla_decode_noalloc", "mla_partial_grid", "mla_debug_inject_stall",
+           "mla_append_kv_fp8", "mla_rope_cos_sin_table", "mla_combine_f32",
+           "mla_merge_rank_partials")
 
 
 class MlaError(RuntimeError):
@@ -74,12 +81,22 @@ def _load_lib():
     lib.mla_decode_partial.restype = i32
     lib.mla_combine.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P]
     lib.mla_combine.restype = i32
-    lib.mla_choose_splits.argtypes = [P, i32, i32, i32, i32, i32, P]
+    lib.mla_choose_splits.argtypes = [P, i32, i32, i32, P]
     lib.mla_choose_splits.restype = i32
     lib.mla_status_string.argtypes = [i32]
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_partial_grid.argtypes = [i32, i32, i32, i32, i32, i32, P]
     lib.mla_partial_grid.restype = i32
+    lib.mla_combine_f32.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P]
+    lib.mla_combine_f32.restype = i32
+    lib.mla_merge_rank_partials.argtypes = [P, P, i32, i32, i32, i32, P, P, P]
+    lib.mla_merge_rank_partials.restype = i32
+    lib.mla_append_kv_fp8.argtypes = [P, P, P, i64, P, i32, P, i32, i32, f32, P, i64, P, P]
+    lib.mla_append_kv_fp8.restype = i32
+    lib.mla_rope_cos_sin_table.argtypes = [P, i64, ctypes.c_double]
+    lib.mla_rope_cos_sin_table.restype = i32
+    lib.mla_device_error_status.argtypes = [i32]
+    lib.mla_device_error_status.restype = i32
     lib.mla_debug_inject_stall.argtypes = [i32]
     lib.mla_debug_inject_stall.restype = i32
     return lib
@@ -180,14 +197,88 @@ def mla_combine(part_o, part_lse, num_splits, max_splits, out, out_lse=None, str
     return out
 
 
-def mla_choose_splits(seq_lens_host, q_len: int, H: int, num_sms: int, max_splits: int):
-    """Per-request split counts (host int32 tensor) for a host list/tensor of seq_lens."""
+def mla_combine_f32(part_o, part_lse, num_splits, max_splits, out_o, out_lse, stream=None):
+    """Merge one rank's split partials into one fp32 partial per row:
+    out_o fp32 [B][q_len][H][512], out_lse fp32 [B][q_len][H]."""
+    B, q_len, H, dl = out_o.shape
+    if dl != 512 or tuple(out_lse.shape) != (B, q_len, H):
+        raise ValueError("out_o must be [B][q_len][H][512] and out_lse [B][q_len][H]")
+    _check("mla_combine_f32", _lib.mla_combine_f32(
+        _dev(part_o, "part_o", torch.float32), _dev(part_lse, "part_lse", torch.float32),
+        _dev(num_splits, "num_splits", torch.int32), int(max_splits), B, q_len, H,
+        _dev(out_o, "out_o", torch.float32), _dev(out_lse, "out_lse", torch.float32),
+        _stream(stream)))
+    return out_o, out_lse
+
+
+def mla_merge_rank_partials(rank_o, rank_lse, out, out_lse=None, stream=None):
+    """Merge per-rank partials rank_o fp32 [N][B][q_len][H][512], rank_lse fp32
+    [N][B][q_len][H] into out bf16 [B][q_len][H][512] (and out_lse)."""
+    N = rank_o.shape[0]
+    B, q_len, H, dl = out.shape
+    if dl != 512 or tuple(rank_o.shape) != (N, B, q_len, H, 512) or \
+            tuple(rank_lse.shape) != (N, B, q_len, H):
+        raise ValueError("rank_o must be [N][B][q_len][H][512], rank_lse [N][B][q_len][H]")
+    _check("mla_merge_rank_partials", _lib.mla_merge_rank_partials(
+        _dev(rank_o, "rank_o", torch.float32), _dev(rank_lse, "rank_lse", torch.float32), N, B,
+        q_len, H, _dev(out, "out", torch.bfloat16),
+        None if out_lse is None else _dev(out_lse, "out_lse", torch.float32), _stream(stream)))
+    return out
+
+
+def mla_choose_splits(seq_lens_host, num_sms: int, max_splits: int):
+    """Per-request split counts (host int32 tensor): one split per 2048 tokens,
+    clamped to [1, max_splits]."""
     sl = torch.as_tensor(seq_lens_host, dtype=torch.int32).contiguous().cpu()
     out = torch.empty_like(sl)
     _check("mla_choose_splits", _lib.mla_choose_splits(
-        ctypes.c_void_p(sl.data_ptr()), sl.numel(), q_len, H, num_sms, max_splits,
+        ctypes.c_void_p(sl.data_ptr()), sl.numel(), num_sms, max_splits,
         ctypes.c_void_p(out.data_ptr())))
     return out
+
+
+def mla_device_error_status(word: int) -> int:
+    """MLA_OK for a zero device error word, MLA_ERR_DEVICE otherwise."""
+    return int(_lib.mla_device_error_status(int(word)))
+
+
+def check_device_error(dev_error) -> None:
+    """Synchronise dev_error's stream and raise MlaError(MLA_ERR_DEVICE) if the
+    GPU set any MLA_DEVERR_* bit."""
+    word = int(dev_error.item())  # .item() waits for the work that writes it
+    _check(f"device error word {word:#x}", mla_device_error_status(word))
+
+
+def mla_rope_cos_sin_table(max_pos: int, base: float = 10000.0) -> torch.Tensor:
+    """Host fp32 [max_pos][32][2] table of (cos, sin) of pos * base^(-2i/64)."""
+    t = torch.empty((max_pos, 32, 2), dtype=torch.float32)
+    _check("mla_rope_cos_sin_table", _lib.mla_rope_cos_sin_table(
+        ctypes.c_void_p(t.data_ptr()), int(max_pos), float(base)))
+    return t
+
+
+def mla_append_kv_fp8(c_kv, k_rope, cos_sin, block_table, seq_lens, inv_scale, kv_pages,
+                      dev_error=None, stream=None):
+    """Write n_new tokens per request into the E4M3 cache kv_pages (uint8
+    [num_pages][64][576]): c_kv bf16 [B][n_new][512], k_rope bf16 [B][n_new][64]
+    (rotated here), cos_sin fp32 [max_pos][32][2] on the device."""
+    B, n_new, dl = c_kv.shape
+    if dl != 512 or tuple(k_rope.shape) != (B, n_new, 64):
+        raise ValueError("c_kv must be [B][n_new][512] and k_rope [B][n_new][64]")
+    if cos_sin.dim() != 3 or tuple(cos_sin.shape[1:]) != (32, 2):
+        raise ValueError("cos_sin must be [max_pos][32][2]")
+    if kv_pages.dim() != 3 or tuple(kv_pages.shape[1:]) != (64, 576):
+        raise ValueError("kv_pages must be [num_pages][64][576]")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B][max_pages]")
+    _check("mla_append_kv_fp8", _lib.mla_append_kv_fp8(
+        _dev(c_kv, "c_kv", torch.bfloat16), _dev(k_rope, "k_rope", torch.bfloat16),
+        _dev(cos_sin, "cos_sin", torch.float32), cos_sin.shape[0],
+        _dev(block_table, "block_table", torch.int32), block_table.shape[1],
+        _dev(seq_lens, "seq_lens", torch.int32), B, n_new, float(inv_scale),
+        _dev(kv_pages, "kv_pages", torch.uint8), kv_pages.shape[0],
+        None if dev_error is None else _dev(dev_error, "dev_error", torch.int32), _stream(stream)))
+    return kv_pages
 
 
 def mla_status_string(status: int) -> str:

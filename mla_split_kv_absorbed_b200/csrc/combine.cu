@@ -12,7 +12,10 @@
 // LSE = M + ln sum w_s.  Grid: (rows, 512 / 128), 128 threads; the split
 // weights of the row are computed once per block into shared memory while the
 // partial loads are in flight.  Up to 256 splits (two per thread for the
-// weights).
+// weights).  The same kernel, with an fp32 output, merges one rank's splits
+// into a single partial per row, and, with the partials laid out one per rank,
+// merges the ranks' partials of a sequence-sharded decode (the same merge one
+// level up).
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -23,36 +26,47 @@ namespace mla {
 constexpr int kCombineThreads = 128;
 constexpr int kCombineGroup = 64;  // partial loads in flight per thread
 
+// Where the partials of a row live: partial s of row r starts at
+// part_o + r * o_row + s * o_split (512 fp32) with its LSE at
+// part_lse[r * l_row + s * l_split].  The split-KV workspace has o_split = 512,
+// o_row = max_splits * 512; partials gathered from several ranks, one per
+// rank, have o_split = rows * 512, o_row = 512.
+struct PartialLayout {
+  int64_t o_row, o_split, l_row, l_split;
+};
+
+template <bool kOutF32>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_lse,
-    const int32_t* __restrict__ num_splits, int max_splits, int rows_per_batch,
-    uint16_t* __restrict__ out, float* __restrict__ out_lse) {
+    const int32_t* __restrict__ num_splits, int splits_const, int max_splits, int rows_per_batch,
+    PartialLayout lay, void* __restrict__ out, float* __restrict__ out_lse) {
   extern __shared__ float w_smem[];  // [max_splits] split weights
   __shared__ float red[2][kCombineThreads / 32];
   const int row = blockIdx.x;
   const int d = blockIdx.y * kCombineThreads + threadIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int b = row / rows_per_batch;
-  int S = num_splits[b];
-  S = S < 0 ? 0 : (S > max_splits ? max_splits : S);
-  const float* po = part_o + (size_t)row * max_splits * 512 + d;
-  const float* pl = part_lse + (size_t)row * max_splits;
+  const float* po = part_o + (int64_t)row * lay.o_row + d;
+  const float* pl = part_lse + (int64_t)row * lay.l_row;
 
-  // launched as a programmatic dependent of the partial kernel: everything
-  // above overlapped its tail; the partials are read only after it completes
+  // launched as a programmatic dependent of the kernel before it on the
+  // stream: everything above overlapped that kernel's tail; memory it may have
+  // written (the partials, and num_splits too) is read only after it completes
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  int S = num_splits != nullptr ? num_splits[b] : splits_const;
+  S = S < 0 ? 0 : (S > max_splits ? max_splits : S);
 
   // issue the first group of partial loads before anything else
   float v[kCombineGroup];
 #pragma unroll
-  for (int j = 0; j < kCombineGroup; ++j) v[j] = (j < S) ? __ldg(po + (size_t)j * 512) : 0.0f;
+  for (int j = 0; j < kCombineGroup; ++j) v[j] = (j < S) ? __ldg(po + (int64_t)j * lay.o_split) : 0.0f;
 
   // split weights while those loads are in flight: M = max LSE, w_s = e^(LSE_s - M)
   float lse[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int sidx = threadIdx.x + k * kCombineThreads;
-    lse[k] = sidx < S ? pl[sidx] : -INFINITY;
+    lse[k] = sidx < S ? pl[(int64_t)sidx * lay.l_split] : -INFINITY;
   }
   float m = fmaxf(lse[0], lse[1]);
 #pragma unroll
@@ -81,7 +95,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     if (g0 > 0) {
 #pragma unroll
       for (int j = 0; j < kCombineGroup; ++j)
-        v[j] = (g0 + j < S) ? __ldg(po + (size_t)(g0 + j) * 512) : 0.0f;
+        v[j] = (g0 + j < S) ? __ldg(po + (int64_t)(g0 + j) * lay.o_split) : 0.0f;
     }
 #pragma unroll
     for (int j = 0; j < kCombineGroup; ++j)
@@ -91,15 +105,19 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
 
   const bool empty = (m == -INFINITY) || !(wsum > 0.0f);
   const float o = empty ? 0.0f : a / wsum;
-  out[(size_t)row * 512 + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+  if (kOutF32)
+    static_cast<float*>(out)[(int64_t)row * 512 + d] = o;
+  else
+    static_cast<uint16_t*>(out)[(int64_t)row * 512 + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
   if (out_lse != nullptr && blockIdx.y == 0 && threadIdx.x == 0)
     out_lse[row] = empty ? -INFINITY : m + logf(wsum);
 }
 
-cudaError_t launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
-                           int max_splits, int B, int q_len, int H, uint16_t* out, float* out_lse,
-                           cudaStream_t stream) {
-  const int rows = B * q_len * H;
+template <bool kOutF32>
+static cudaError_t launch_combine_any(const float* part_o, const float* part_lse,
+                                      const int32_t* num_splits, int splits_const, int max_splits,
+                                      int rows, int rows_per_batch, const PartialLayout& lay,
+                                      void* out, float* out_lse, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, 512 / kCombineThreads);
@@ -107,14 +125,37 @@ cudaError_t launch_combine(const float* part_o, const float* part_lse, const int
   cfg.dynamicSmemBytes = sizeof(float) * (size_t)max_splits;
   cfg.stream = stream;
   // programmatic dependent launch: the grid may be scheduled while the
-  // partial kernel before it on the stream is still running
+  // kernel before it on the stream is still running
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, part_o, part_lse, num_splits, max_splits,
-                            q_len * H, out, out_lse);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<kOutF32>, part_o, part_lse, num_splits,
+                            splits_const, max_splits, rows_per_batch, lay, out, out_lse);
+}
+
+cudaError_t launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                           int max_splits, int B, int q_len, int H, uint16_t* out, float* out_lse,
+                           cudaStream_t stream) {
+  const PartialLayout lay = {(int64_t)max_splits * 512, 512, max_splits, 1};
+  return launch_combine_any<false>(part_o, part_lse, num_splits, 0, max_splits, B * q_len * H,
+                                   q_len * H, lay, out, out_lse, stream);
+}
+
+cudaError_t launch_combine_f32(const float* part_o, const float* part_lse,
+                               const int32_t* num_splits, int max_splits, int B, int q_len, int H,
+                               float* out, float* out_lse, cudaStream_t stream) {
+  const PartialLayout lay = {(int64_t)max_splits * 512, 512, max_splits, 1};
+  return launch_combine_any<true>(part_o, part_lse, num_splits, 0, max_splits, B * q_len * H,
+                                  q_len * H, lay, out, out_lse, stream);
+}
+
+cudaError_t launch_merge_ranks(const float* rank_o, const float* rank_lse, int n_ranks, int rows,
+                               uint16_t* out, float* out_lse, cudaStream_t stream) {
+  const PartialLayout lay = {512, (int64_t)rows * 512, 1, rows};
+  return launch_combine_any<false>(rank_o, rank_lse, nullptr, n_ranks, n_ranks, rows, rows, lay,
+                                   out, out_lse, stream);
 }
 
 }  // namespace mla

@@ -568,14 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap& kv_map,
                                cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(bf16k::decode_bf16_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         bf16k::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // the shared-memory opt-in is a per-device attribute of the kernel: set it
+  // on every launch (a cheap host call) so that any device the caller makes
+  // current is configured
+  cudaError_t e = cudaFuncSetAttribute(bf16k::decode_bf16_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bf16k::kSmemBytes);
+  if (e != cudaSuccess) return e;
   const int groups = (a.q_len * a.H + bf16k::kRows - 1) / bf16k::kRows;
   dim3 grid(groups, a.max_splits, a.B);
   bf16k::decode_bf16_kernel<<<grid, bf16k::kThreads, bf16k::kSmemBytes, stream>>>(a, kv_map);

@@ -11,6 +11,7 @@
 // The cost: every process that loads the library holds kScratchRowSplits *
 // 513 * 4 bytes (about 16 MiB) of device memory on each GPU it uses, until
 // the process exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -29,8 +30,45 @@ constexpr int64_t kScratchRowSplits = 8192;
 static __device__ __align__(256) float g_partials_scratch[kScratchRowSplits * 513];
 
 constexpr int kMaxDevices = 64;
-float* g_scratch_ptr[kMaxDevices] = {};
+
+// The cached address is tagged with the CUDA context it was looked up in: a
+// context that is destroyed and created again (cudaDeviceReset, a primary
+// context released and retained again) reloads the module, and the array may
+// then live elsewhere, so a changed context id triggers a new look-up.
+struct ScratchEntry {
+  float* ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+ScratchEntry g_scratch[kMaxDevices];
 std::mutex g_scratch_mutex;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (0 if it cannot be had).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_partials_scratch on the current device.  In host code
 // the symbol's name is only a host-side stand-in; the address the kernels
@@ -40,13 +78,19 @@ int scratch_for_current_device(float** out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MLA_ERR_CUDA;
   if (dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  // (before the device's first runtime call there is no current context and
+  // the id is 0: the look-up below creates the context and is repeated once
+  // on the next call, which then finds the context's id)
+  const unsigned long long ctx = current_context_id();
+  ScratchEntry& e = g_scratch[dev];
+  if (e.ptr == nullptr || ctx == 0 || e.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_partials_scratch) != cudaSuccess || p == nullptr)
       return MLA_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<float*>(p);
+    e.ptr = static_cast<float*>(p);
+    e.ctx_id = ctx;
   }
-  *out = g_scratch_ptr[dev];
+  *out = e.ptr;
   return MLA_OK;
 }
 

@@ -12,6 +12,13 @@ cudaError_t launch_quantize_fp8(const uint16_t* x, uint8_t* y, int64_t n, float 
 cudaError_t launch_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,
                            int max_splits, int B, int q_len, int H, uint16_t* out, float* out_lse,
                            cudaStream_t stream);
+// The same merge with an fp32 output: one partial per row (O [rows][512], LSE).
+cudaError_t launch_combine_f32(const float* part_o, const float* part_lse,
+                               const int32_t* num_splits, int max_splits, int B, int q_len, int H,
+                               float* out, float* out_lse, cudaStream_t stream);
+// Merge of per-rank partials laid out [n_ranks][rows][512] and [n_ranks][rows].
+cudaError_t launch_merge_ranks(const float* rank_o, const float* rank_lse, int n_ranks, int rows,
+                               uint16_t* out, float* out_lse, cudaStream_t stream);
 
 // Arguments of the split-KV partial kernels (device pointers; see mla.h).
 struct DecodeArgs {
@@ -52,5 +59,24 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cu
 // 1 page}, 128-byte swizzle.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, const CUtensorMap& kv_map,
                                cudaStream_t stream);
+
+// Arguments of the KV-append kernel (device pointers; see mla.h).
+struct AppendArgs {
+  const uint16_t* c_kv;        // [B][n_new][512] bf16
+  const uint16_t* k_rope;      // [B][n_new][64] bf16, before rotation
+  const float* cos_sin;        // [max_pos][32][2] fp32
+  const int32_t* block_table;  // [B][max_pages]
+  const int32_t* seq_lens;     // [B], including the n_new tokens
+  uint8_t* kv_pages;           // [num_pages][64][576] E4M3
+  int32_t* dev_error;
+  int64_t max_pos;
+  int64_t num_pages;
+  int max_pages;
+  int B;
+  int n_new;
+  float inv_scale;
+};
+
+cudaError_t launch_append_kv_fp8(const AppendArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace mla

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 
 #include "kernels.cuh"
@@ -18,20 +19,27 @@ std::atomic<int> g_inject_stall{0};  // mla_debug_inject_stall
 
 constexpr int kPage = 64;
 constexpr int kRow = 576;
+constexpr int kSplitTokens = 2048;  // mla_choose_splits: tokens per split
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int num_sms_cached() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-      return 148;
-    sms = v;
+// SM count of the current device, looked up once per device (the partial
+// kernel's grid plan depends on it; a process may drive several devices).
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_num_sms[kMaxDevices] = {};
+
+int num_sms_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < kMaxDevices) {
+    const int cached = g_num_sms[dev].load(std::memory_order_relaxed);
+    if (cached > 0) return cached;
   }
-  return sms;
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    return 148;
+  if (dev < kMaxDevices) g_num_sms[dev].store(v, std::memory_order_relaxed);
+  return v;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -116,7 +124,7 @@ int mla_quantize_fp8(const uint16_t* x_bf16, uint8_t* y_e4m3, int64_t n, float i
   if (n < 0) return MLA_ERR_INVALID_ARG;
   if (n == 0) return MLA_OK;
   if (x_bf16 == nullptr || y_e4m3 == nullptr) return MLA_ERR_INVALID_ARG;
-  return status_of(mla::launch_quantize_fp8(x_bf16, y_e4m3, n, inv_scale, num_sms_cached(),
+  return status_of(mla::launch_quantize_fp8(x_bf16, y_e4m3, n, inv_scale, num_sms_current_device(),
                                             static_cast<cudaStream_t>(stream)));
 }
 
@@ -146,7 +154,7 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   if (!(softmax_scale == softmax_scale) || !(kv_scale == kv_scale) || kv_scale <= 0.0f)
     return MLA_ERR_INVALID_ARG;
   if (kv_dtype == MLA_KV_BF16 && kv_scale != 1.0f) return MLA_ERR_INVALID_ARG;
-  if (q_len > 4 || H > 128 || max_splits > 256 || B > 65535 || (q_len * H) % 16 != 0)
+  if (q_len > 4 || q_len * H > 512 || max_splits > 256 || B > 65535 || (q_len * H) % 16 != 0)
     return MLA_ERR_UNSUPPORTED;
 
   CUtensorMap map;
@@ -175,7 +183,7 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   a.inject_stall = g_inject_stall.load(std::memory_order_relaxed);
   {
     int32_t plan[4];
-    plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms_cached(), plan);
+    plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms_current_device(), plan);
     a.groups = (q_len * H + 63) / 64;
     a.pieces = plan[1];
     a.split_from = plan[2];
@@ -192,32 +200,95 @@ int mla_combine(const float* part_o, const float* part_lse, const int32_t* num_s
   if (part_o == nullptr || part_lse == nullptr || num_splits == nullptr || out_bf16 == nullptr)
     return MLA_ERR_INVALID_ARG;
   if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return MLA_ERR_INVALID_ARG;
-  if (max_splits > 256 || q_len > 4 || H > 128) return MLA_ERR_UNSUPPORTED;
+  if (max_splits > 256 || q_len > 4 || q_len * H > 512) return MLA_ERR_UNSUPPORTED;
   return status_of(mla::launch_combine(part_o, part_lse, num_splits, max_splits, B, q_len, H,
                                        out_bf16, out_lse, static_cast<cudaStream_t>(stream)));
 }
 
-int mla_choose_splits(const int32_t* seq_lens_host, int B, int q_len, int H, int num_sms,
-                      int max_splits, int32_t* out_host) {
-  if (seq_lens_host == nullptr || out_host == nullptr || B <= 0 || q_len <= 0 || H <= 0 ||
-      num_sms <= 0 || max_splits <= 0)
+int mla_combine_f32(const float* part_o, const float* part_lse, const int32_t* num_splits,
+                    int max_splits, int B, int q_len, int H, float* out_o, float* out_lse,
+                    void* stream) {
+  if (part_o == nullptr || part_lse == nullptr || num_splits == nullptr || out_o == nullptr ||
+      out_lse == nullptr)
     return MLA_ERR_INVALID_ARG;
-  const int groups = (q_len * H + 63) / 64;
-  int64_t total_pages = 0;
+  if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return MLA_ERR_INVALID_ARG;
+  if (max_splits > 256 || q_len > 4 || q_len * H > 512) return MLA_ERR_UNSUPPORTED;
+  return status_of(mla::launch_combine_f32(part_o, part_lse, num_splits, max_splits, B, q_len, H,
+                                           out_o, out_lse, static_cast<cudaStream_t>(stream)));
+}
+
+int mla_merge_rank_partials(const float* rank_o, const float* rank_lse, int n_ranks, int B,
+                            int q_len, int H, uint16_t* out_bf16, float* out_lse, void* stream) {
+  if (rank_o == nullptr || rank_lse == nullptr || out_bf16 == nullptr) return MLA_ERR_INVALID_ARG;
+  if (n_ranks <= 0 || B <= 0 || q_len <= 0 || H <= 0) return MLA_ERR_INVALID_ARG;
+  if (n_ranks > 256 || q_len > 4 || q_len * H > 512) return MLA_ERR_UNSUPPORTED;
+  const int64_t rows = (int64_t)B * q_len * H;
+  if (rows > 0x7FFFFFFF) return MLA_ERR_UNSUPPORTED;
+  return status_of(mla::launch_merge_ranks(rank_o, rank_lse, n_ranks, (int)rows, out_bf16, out_lse,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int mla_choose_splits(const int32_t* seq_lens_host, int B, int num_sms, int max_splits,
+                      int32_t* out_host) {
+  if (seq_lens_host == nullptr || out_host == nullptr || B <= 0 || num_sms <= 0 || max_splits <= 0)
+    return MLA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (seq_lens_host[b] < 1) return MLA_ERR_INVALID_ARG;
+  // one split per 2048 tokens (32 pages), at least one, at most max_splits
   for (int b = 0; b < B; ++b) {
-    if (seq_lens_host[b] < q_len) return MLA_ERR_INVALID_ARG;
-    total_pages += (seq_lens_host[b] + kPage - 1) / kPage;
-  }
-  // about two waves of (request, split, row-group) CTAs, at least 16 pages each
-  const int64_t target_ctas = 2 * (int64_t)num_sms;
-  int64_t pages_per_split = (total_pages * groups + target_ctas - 1) / target_ctas;
-  if (pages_per_split < 16) pages_per_split = 16;
-  for (int b = 0; b < B; ++b) {
-    const int64_t pages = (seq_lens_host[b] + kPage - 1) / kPage;
-    int64_t sp = (pages + pages_per_split - 1) / pages_per_split;
+    int64_t sp = ((int64_t)seq_lens_host[b] + kSplitTokens - 1) / kSplitTokens;
     if (sp < 1) sp = 1;
     if (sp > max_splits) sp = max_splits;
     out_host[b] = (int32_t)sp;
+  }
+  return MLA_OK;
+}
+
+int mla_device_error_status(int32_t dev_error_word) {
+  return dev_error_word == 0 ? MLA_OK : MLA_ERR_DEVICE;
+}
+
+int mla_append_kv_fp8(const uint16_t* c_kv, const uint16_t* k_rope, const float* cos_sin,
+                      int64_t max_pos, const int32_t* block_table, int max_pages_per_req,
+                      const int32_t* seq_lens, int B, int n_new, float inv_scale, uint8_t* kv_pages,
+                      int64_t num_pages, int32_t* dev_error, void* stream) {
+  if (B <= 0 || n_new < 0 || max_pos <= 0 || max_pages_per_req <= 0 || num_pages <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (n_new == 0) return MLA_OK;
+  if (c_kv == nullptr || k_rope == nullptr || cos_sin == nullptr || block_table == nullptr ||
+      seq_lens == nullptr || kv_pages == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(c_kv) || !aligned16(kv_pages) || (reinterpret_cast<uintptr_t>(k_rope) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(cos_sin) & 7u) != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!(inv_scale == inv_scale) || !(inv_scale > 0.0f)) return MLA_ERR_INVALID_ARG;
+  mla::AppendArgs a = {};
+  a.c_kv = c_kv;
+  a.k_rope = k_rope;
+  a.cos_sin = cos_sin;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.kv_pages = kv_pages;
+  a.dev_error = dev_error;
+  a.max_pos = max_pos;
+  a.num_pages = num_pages;
+  a.max_pages = max_pages_per_req;
+  a.B = B;
+  a.n_new = n_new;
+  a.inv_scale = inv_scale;
+  return status_of(mla::launch_append_kv_fp8(a, num_sms_current_device(),
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int mla_rope_cos_sin_table(float* cos_sin_host, int64_t max_pos, double base) {
+  if (cos_sin_host == nullptr || max_pos <= 0 || !(base > 1.0)) return MLA_ERR_INVALID_ARG;
+  for (int64_t pos = 0; pos < max_pos; ++pos) {
+    for (int i = 0; i < 32; ++i) {
+      // theta_i = base^(-2i/64); angle, cosine and sine in double, rounded once
+      const double angle = (double)pos * std::pow(base, -(double)(2 * i) / 64.0);
+      cos_sin_host[(pos * 32 + i) * 2] = (float)std::cos(angle);
+      cos_sin_host[(pos * 32 + i) * 2 + 1] = (float)std::sin(angle);
+    }
   }
   return MLA_OK;
 }

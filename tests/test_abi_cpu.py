@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -25,11 +26,15 @@ def header_functions():
 
 def test_header_declares_the_entry_points():
     names = header_functions()
-    assert set(names) == {"mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
-                          "mla_combine", "mla_choose_splits", "mla_status_string"} | (
-        set(names) - {"mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
-                      "mla_combine", "mla_choose_splits", "mla_status_string"})
+    required = {"mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
+                "mla_combine", "mla_choose_splits", "mla_status_string", "mla_device_error_status"}
+    assert required <= set(names)
     assert len(names) == len(set(names))
+
+
+def test_binding_exports_match_header():
+    import mla_split_kv_absorbed_b200 as m
+    assert set(m.EXPORTS) == set(header_functions())
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -53,20 +58,35 @@ def test_status_strings(lib):
     assert lib.status_string(99) == "MLA_ERR_UNKNOWN"
 
 
-def test_choose_splits(lib):
-    # batch 1 at 128K on 148 SMs: enough splits for about two waves
-    s1 = lib.mla_choose_splits([131072], 1, 64, 148, 64)
-    assert s1.tolist() == [64]
-    s16 = lib.mla_choose_splits([131072] * 16, 1, 64, 148, 64)
-    assert all(v == s16[0] for v in s16.tolist()) and 8 <= int(s16[0]) <= 64
-    # short requests get one split, never more than max_splits, never zero
+def test_choose_splits_follows_the_length_rule(lib):
+    # the reading the ragged workload uses: one split per 2048 tokens, 1..max_splits
+    from mla_split_kv_absorbed_b200 import workloads as wl
+    rng = np.random.default_rng(7)
+    lens = np.concatenate([[1, 2047, 2048, 2049, 4096, 131072, 262144, 1 << 30],
+                           rng.integers(1, 300000, size=500)]).astype(np.int32)
+    got = lib.mla_choose_splits(lens, 148, 64).numpy()
+    want = np.array([wl.splits_by_length(int(L)) for L in lens])
+    assert np.array_equal(got, want)
+    # the formula itself, written out: ceil(L / 2048) clamped to [1, max_splits]
+    for max_splits in (1, 7, 64, 256):
+        got = lib.mla_choose_splits(lens, 148, max_splits).numpy()
+        assert np.array_equal(got, np.clip(-(-lens.astype(np.int64) // 2048), 1, max_splits))
+    assert lib.mla_choose_splits([131072], 148, 64).tolist() == [64]  # the batch-1 64-way split
+    # the SM count does not change the rule
+    assert np.array_equal(lib.mla_choose_splits(lens, 1, 64).numpy(),
+                          lib.mla_choose_splits(lens, 148, 64).numpy())
     with pytest.raises(lib.MlaError):
-        lib.mla_choose_splits([1], 4, 64, 148, 64)  # seq_len below q_len
-    s = lib.mla_choose_splits([4, 64, 1000, 262144], 4, 64, 148, 64).tolist()
-    assert s[0] == 1 and s[1] == 1 and 1 <= s[2] <= 64 and s[3] <= 64
-    # at least 16 pages per split
-    s = lib.mla_choose_splits([64 * 16 * 5], 1, 16, 148, 256).tolist()
-    assert s == [5]
+        lib.mla_choose_splits([0], 148, 64)  # empty request
+    with pytest.raises(lib.MlaError):
+        lib.mla_choose_splits([10], 0, 64)
+
+
+def test_device_error_status(lib):
+    assert lib.mla_device_error_status(0) == lib.MLA_OK
+    for bit in (lib.DEVERR_BAD_PAGE, lib.DEVERR_BAD_SEQLEN, lib.DEVERR_TIMEOUT,
+                lib.DEVERR_BAD_SPLITS, lib.DEVERR_SMEM_ALIGN, 0x7FFFFFFF, -1):
+        assert lib.mla_device_error_status(bit) == lib.MLA_ERR_DEVICE
+    assert lib.status_string(lib.MLA_ERR_DEVICE) == "MLA_ERR_DEVICE"
 
 
 def test_rejections_without_gpu(lib):
@@ -78,13 +98,14 @@ def test_rejections_without_gpu(lib):
     assert h.mla_combine(null, null, null, 1, 1, 1, 64, null, null, null) == lib.MLA_ERR_INVALID_ARG
     assert h.mla_quantize_fp8(null, null, -1, 1.0, null) == lib.MLA_ERR_INVALID_ARG
     assert h.mla_quantize_fp8(null, null, 0, 1.0, null) == lib.MLA_OK  # n = 0 is a no-op
-    assert h.mla_choose_splits(null, 1, 1, 64, 148, 64, null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_choose_splits(null, 1, 148, 64, null) == lib.MLA_ERR_INVALID_ARG
     # unsupported shapes are reported as such (fake but aligned non-null pointers: nothing launches)
     fake = ctypes.c_void_p(1 << 20)
     args = [fake, fake, fake, 0, 1.0, 10, fake, 4, fake, fake, 4, 1]
     assert h.mla_decode_partial(*args, 5, 64, 1.0, fake, fake, null, null) == lib.MLA_ERR_UNSUPPORTED  # q_len 5
     assert h.mla_decode_partial(*args, 1, 24, 1.0, fake, fake, null, null) == lib.MLA_ERR_UNSUPPORTED  # H*q_len % 16
-    assert h.mla_decode_partial(*args, 1, 256, 1.0, fake, fake, null, null) == lib.MLA_ERR_UNSUPPORTED  # H > 128
+    assert h.mla_decode_partial(*args, 1, 528, 1.0, fake, fake, null, null) == lib.MLA_ERR_UNSUPPORTED  # rows > 512
+    assert h.mla_decode_partial(*args, 4, 144, 1.0, fake, fake, null, null) == lib.MLA_ERR_UNSUPPORTED  # q_len*H > 512
     # bad kv_dtype / bf16 with kv_scale != 1 / non-positive scale
     a2 = [fake, fake, fake, 7, 1.0, 10, fake, 4, fake, fake, 4, 1, 1, 64, 1.0, fake, fake, null, null]
     assert h.mla_decode_partial(*a2) == lib.MLA_ERR_INVALID_ARG
@@ -127,3 +148,33 @@ def test_partial_grid_plan(lib):
     assert m.mla_partial_grid(1, 1, 16, 4, BF16, 148)[0] == 4
     with pytest.raises(m.MlaError):
         m.mla_partial_grid(0, 1, 64, 4, FP8, 148)
+
+
+def test_rope_table_matches_the_oracle_bit_for_bit(lib, oracle_lib):
+    # the library's host table builder and the oracle's are separate code for
+    # the same definition (angle, cosine and sine in double, rounded once)
+    t_lib = lib.mla_rope_cos_sin_table(5000).numpy()
+    t_ora = oracle_lib.rope_table(5000)
+    assert np.array_equal(t_lib, t_ora)
+    assert np.array_equal(lib.mla_rope_cos_sin_table(70, 500000.0).numpy(),
+                          oracle_lib.rope_table(70, 500000.0))
+    with pytest.raises(lib.MlaError):
+        lib.mla_rope_cos_sin_table(0)
+
+
+def test_append_rejections_without_gpu(lib):
+    h = lib.load()
+    null = None
+    fake = ctypes.c_void_p(1 << 20)
+    # null pointers, bad sizes, misalignment, bad scale: rejected before any launch
+    assert h.mla_append_kv_fp8(null, fake, fake, 10, fake, 4, fake, 1, 1, 1.0, fake, 10, null,
+                               null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_append_kv_fp8(fake, fake, fake, 10, fake, 4, fake, 0, 1, 1.0, fake, 10, null,
+                               null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_append_kv_fp8(ctypes.c_void_p((1 << 20) + 8), fake, fake, 10, fake, 4, fake, 1, 1,
+                               1.0, fake, 10, null, null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_append_kv_fp8(fake, fake, fake, 10, fake, 4, fake, 1, 1, -1.0, fake, 10, null,
+                               null) == lib.MLA_ERR_INVALID_ARG
+    # nothing to append is a no-op
+    assert h.mla_append_kv_fp8(null, null, null, 10, null, 4, null, 1, 0, 1.0, null, 10, null,
+                               null) == lib.MLA_OK

@@ -137,13 +137,21 @@ FULL = [("b1_128k_fp8", 64), ("b16_128k_fp8", 32), ("verify_q4_256k_fp8", 24),
 
 @pytest.mark.parametrize("spec,n_rows", FULL)
 def test_decode_full_size_sampled_rows(spec, n_rows):
+    # Benchmark workloads in the benchmark's launch configuration.  The rows
+    # compared are the first and last, one seeded row of every request (so
+    # every request's splits, including the units of a cut last wave, feed a
+    # compared row) and n_rows more seeded rows.
     c = make_case(spec, gen_device="cuda")
     w = c.w
     out, lse, _, _, err = run_gpu(c)
     assert err == 0
     R = w.B * w.q_len * w.H
+    per_req = w.q_len * w.H
     rng = np.random.default_rng(123)
-    rows = np.unique(np.concatenate([[0, R - 1], rng.choice(R, size=min(n_rows, R), replace=False)]))
+    one_per_request = np.arange(w.B) * per_req + rng.integers(0, per_req, size=w.B)
+    rows = np.unique(np.concatenate([[0, R - 1], one_per_request,
+                                     rng.choice(R, size=min(n_rows, R), replace=False)]))
+    assert len(np.unique(rows // per_req)) == w.B
     o_ref, l_ref = oracle_rows(c, rows)
     o = out.float().cpu().numpy().reshape(R, 512)[rows]
     l = lse.cpu().numpy().reshape(R)[rows]

@@ -16,14 +16,21 @@ from gpu_helpers import assert_attention_close, make_case, oracle_rows, run_gpu
 
 pytestmark = pytest.mark.gpu
 
-# 128 splits of one page each: the grid fills more than half of the SMs, so
-# every split is one CTA (no cluster), and CTA (0, 0, 0) is split 0.
-CASE = ("b1_128k_fp8", dict(seq_lens=[8192], splits=128))
+CASES = [
+    # 128 splits of one page each: the grid fills more than half of the SMs,
+    # so every split is one CTA (no cluster), and CTA 0 is split 0
+    ("b1_128k_fp8", dict(seq_lens=[8192], splits=128)),
+    # 4 splits: every split is cut into 4 pieces (clusters of 4 CTAs that
+    # merge through distributed shared memory); CTA 0 is piece 0 of split 0,
+    # and its peers wait for it at the cluster barrier
+    ("b1_128k_fp8", dict(seq_lens=[8192], splits=4)),
+]
 
 
-def test_stalled_load_times_out_and_context_survives():
+@pytest.mark.parametrize("case", CASES, ids=["one-cta-units", "cluster-cut-units"])
+def test_stalled_load_times_out_and_context_survives(case):
     import mla_split_kv_absorbed_b200 as m
-    c = make_case(CASE[0], **CASE[1])
+    c = make_case(case[0], **case[1])
     w = c.w
     part_o, part_lse = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")

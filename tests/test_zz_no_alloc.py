@@ -13,7 +13,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import LSE_TOL, O_MAX_ABS, O_REL_L2, bf16_half_ulp, make_case, run_gpu
+from gpu_helpers import (LSE_TOL, O_MAX_ABS, O_REL_L2, assert_attention_close, bf16_half_ulp,
+                         make_case, oracle_rows, run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -64,6 +65,28 @@ def test_noalloc_matches_partial_plus_combine_on_two_calls_in_a_row():
         assert st == m.MLA_OK, m.status_string(st)
         assert err == 0 and ref_err == 0
         _assert_close(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("spec,ov", [
+    # bf16 cache through the shared scratch
+    ("tiny", dict(seq_lens=[777, 2000], splits=3, H=64)),
+    # FP8, 128 splits x 64 heads = the whole scratch; more than half the SMs
+    # are busy, so every split is one CTA (no cluster)
+    ("b1_128k_fp8", dict(seq_lens=[16384], splits=128)),
+])
+def test_noalloc_matches_the_oracle(spec, ov):
+    import mla_split_kv_absorbed_b200 as m
+    lib = m.load()
+    c = make_case(spec, **ov)
+    w = c.w
+    for _ in range(2):  # the second call reuses scratch the first one filled
+        st, out, lse, err = _noalloc(lib, c)
+        assert st == m.MLA_OK, m.status_string(st)
+        assert err == 0
+        rows = np.arange(w.B * w.q_len * w.H)
+        o_ref, l_ref = oracle_rows(c, rows)
+        assert_attention_close(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
+                               o_ref, l_ref, what=f"noalloc {spec}")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
