@@ -16,50 +16,55 @@
 // that merges its results on chip (merge_pieces) - all units when they fill at
 // most half of the GPU, or only those of a partly filled last wave.
 //
-// Tensor-core mapping (tokens as M): with at most 64 query rows per CTA,
-// using the rows as M would run the half-width M=64 UMMA shape and would need
-// a 64x512 fp32 O accumulator beside S, which does not fit TMEM.  Instead the
-// 128 tokens of a tile are M=128:
-//   S^T[t][n] = K[t][:] . Q[n][:]        A = K tile (K-major), B = Q (K-major)
-//   O^T[d][n] += V^T[d][t] . P[t][n]     A = V tile (MN-major), B = P (MN-major)
-// for d in four 128-wide blocks of the 512 latent dims.  V is the first 512
-// columns of the same resident tile that fed K, so every KV byte crosses HBM
-// once and shared memory once.
-//
 // Exact two-term FP8 operands: the cache is E4M3, and kind::f8f6f4 needs both
 // operands E4M3.  Q (bf16, 8 significant bits) is scaled per row by a power
 // of two and split as Q = Q_hi + Q_lo with Q_hi = Q rounded to 4 significant
 // bits and Q_lo = E4M3(Q - Q_hi); this is exact for every element within a
-// factor 2^-9 of the row maximum (smaller ones carry an absolute error of at
-// most 2^-16 of the maximum).  B = [Q_hi ; Q_lo] is one N=128 operand, so S_hi and S_lo
-// come out of one MMA and the softmax adds them.  The softmax weights are
-// scaled by 2^7, p' = 2^(s - m + 7), and split the same way, P = P_hi + P_lo:
-// about 8 significant bits (like bf16) for every p' >= 2^-2 and an absolute
-// error of at most 2^-9 for smaller weights.  PV accumulates both terms; the scale
-// cancels in O / l and is removed from the LSE.
+// factor 2^-9 of the row maximum.  The softmax weights are scaled by 2^7,
+// p' = 2^(s - m + 7), and split the same way, P = P_hi + P_lo: about 8
+// significant bits (like bf16) for every p' >= 2^-2 and an absolute error of
+// at most 2^-9 for smaller weights.  The scale cancels in O / l and is removed
+// from the LSE.
+//
+// Tensor-core mapping.  QK^T takes the 128 two-term query rows as M and the
+// 128 tokens of a tile as N:
+//   S'[m][t] = Q'[m][:] . K[t][:]      A = Q' (tensor memory for the 512
+//                                      latent dims, shared memory for the 64
+//                                      RoPE dims), B = K tile (K-major)
+// Row m = 32 qd + l of Q' (qd = TMEM lane quadrant, l = lane) is query row
+// n = 16 qd + (l & 15), term hi for l < 16 and lo for l >= 16, so the two
+// terms of a score sit in lanes l and l ^ 16 of one warp and are added with
+// one shuffle.  Keeping the 512 latent dims of Q' in tensor memory frees 64
+// KiB of shared memory for the KV ring.  PV keeps the tokens as K and the
+// latent dims as M (a 64 x 512 fp32 O with rows as M would not fit in tensor
+// memory beside S'):
+//   O^T[d][n] += V^T[d][t] . P[t][n]   A = V tile (MN-major), B = P (K-major)
+// for d in four 128-wide blocks; the hi and lo MMAs of one block and K step
+// share A through the MMA's A-operand collector, so V is read from shared
+// memory once.  V is the first 512 columns of the same resident tile that fed
+// K, so every KV byte crosses HBM once.
 //
 // Online softmax (log2 domain, scores pre-multiplied by log2 e), with a lazy
 // running max: the max m used for a row only moves when a tile's max exceeds
 // it by more than 1.75 (log2 units), so p' stays <= 2^8.75 < 448, the E4M3
-// maximum, and rescaling of the O^T columns and row sums (by
-// 2^(m_old - m_new)) is rare.  A tile whose max moved nowhere does not wait
-// for the previous tile's PV before its own PV is released.
+// maximum.  A tile in which no score of a quadrant's rows exceeds its max by
+// that much (the common case once the max has settled) skips the max
+// reduction altogether: one barrier vote decides it.  O^T columns and row
+// sums are rescaled (by 2^(m_old - m_new)) only for rows whose max moved.
 //
 // Warp roles (768 threads):
-//   warp 0        TMA producer: pages -> 64-byte-swizzled chunks, plus L2
-//                 prefetch of tiles up to three ahead
-//   warp 1        UMMA issuer (warp-uniform polling of readiness, so a ready
-//                 PV is never held behind QK data still in flight; one
-//                 elected lane issues) and TMEM owner
-//   warps 4-19    softmax in four warpgroups of 16 query columns each
-//                 (thread = token row of S^T); the softmax of a tile is on
-//                 the critical path of the two-tile ring, so it gets the
-//                 most warps that the register file allows
+//   warp 0        TMA producer: pages -> 64-byte-swizzled 128-dim pairs in an
+//                 11-slot ring (2.75 tiles) plus a 2-slot RoPE ring, and L2
+//                 prefetch of tiles ahead
+//   warp 1        UMMA issuer (warp-uniform polling of readiness, PV before
+//                 QK; one elected lane issues) and TMEM owner
+//   warps 4-19    softmax: warp w works on TMEM lane quadrant w % 4 (16 query
+//                 rows) and token slice (w - 4) / 4 (32 tokens of the tile)
 //   warps 20-23   O^T rescaling between tiles (thread = latent dim)
 //   warps 4-23    epilogue: O^T / l from TMEM to the partial output
 //   warps 4-19    also convert Q to the split FP8 operand at the start
-// TMEM (512 columns): S^T buffers at 0 and 128 (S_hi 0-63 | S_lo 64-127),
-// O^T blocks at 256 + 64*j.
+// TMEM (512 columns): O^T blocks at 64 j (0-255), Q' latent at 256-383, S' at
+// 384-511.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -71,61 +76,70 @@ namespace mla {
 namespace fp8k {
 
 constexpr int kThreads = 768;
-constexpr int kSoftGroups = 4;      // softmax warpgroups
-constexpr int kCols = 16;           // query columns per softmax warpgroup
-constexpr int kSoftThreads = 128 * kSoftGroups;
+constexpr int kSoftWarps = 16;
+constexpr int kSoftThreads = 32 * kSoftWarps;
 constexpr int kRows = 64;           // query rows per CTA (UMMA N for PV)
-constexpr int kTile = 128;          // tokens per tile (UMMA M)
+constexpr int kTile = 128;          // tokens per tile (UMMA N for QK, K for PV)
 constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
 constexpr uint32_t kPageBytes = 64 * 576;  // one page of the pool
-constexpr int kRingPairs = 8;       // two tiles of latent dims in flight
+constexpr int kRingPairs = 11;      // latent pair slots: 2.75 tiles in flight
+constexpr int kRopeSlots = 2;
 constexpr float kPShift = 7.0f;     // log2 of the factor carried by the softmax weights
-constexpr float kLazy = 1.75f;       // the used max moves only when exceeded by more than this
+constexpr float kLazy = 1.75f;      // the used max moves only when exceeded by more than this
 
-constexpr int kOffQ = 0;                                 // 9 chunks, rows hi 0-63 | lo 64-127
-constexpr int kOffRing = kOffQ + 9 * kChunk;             // 73728
-constexpr int kOffRope = kOffRing + kRingPairs * kPair;  // 204800
-constexpr int kOffPhi = kOffRope + kChunk;               // 212992
-constexpr int kOffPlo = kOffPhi + kChunk;                // 221184
-constexpr int kOffScratch = kOffPlo + kChunk;            // 229376
-constexpr int kSmemBytes = 232448;                       // 227 KiB
+constexpr int kOffRing = 0;                                  // 11 pairs
+constexpr int kOffRope = kOffRing + kRingPairs * kPair;      // 180224: 2 RoPE chunks
+constexpr int kOffQr = kOffRope + kRopeSlots * kChunk;       // 196608: Q' RoPE dims [128][64 B]
+constexpr int kOffPhi = kOffQr + kChunk;                     // 204800: P_hi [64 rows][128 B]
+constexpr int kOffPlo = kOffPhi + kChunk;                    // 212992: P_lo
+constexpr int kOffScratch = kOffPlo + kChunk;                // 221184
+constexpr int kSmemBytes = 232448;                           // 227 KiB
+
+constexpr uint32_t kTmemO = 0;      // O^T block j at 64 j
+constexpr uint32_t kTmemQ = 256;    // Q' latent dims: K step k at 256 + 8 k
+constexpr uint32_t kTmemS = 384;    // S' [128 rows][128 tokens]
 
 // barrier indices
-constexpr int kBarNopeFull = 0;    // 8
-constexpr int kBarNopeEmpty = 8;   // 8
-constexpr int kBarRopeFull = 16;
-constexpr int kBarRopeEmpty = 17;
-constexpr int kBarSFull = 18;      // 2
-constexpr int kBarSEmpty = 20;     // 2
-constexpr int kBarPFull = 22;
-constexpr int kBarPEmpty = 23;
-constexpr int kBarOReady = 24;     // 2: per tile parity (the rescale loop may run a tile ahead)
-constexpr int kBarPvDone = 26;
-constexpr int kBarQReady = 27;
-constexpr int kBarAlphaFull = 28;  // 2: per tile parity (the softmax groups may be a tile apart)
-constexpr int kBarDrain = 30;
+constexpr int kBarFull = 0;                      // 11
+constexpr int kBarEmpty = kBarFull + kRingPairs;  // 11
+constexpr int kBarRopeFull = 22;   // 2
+constexpr int kBarRopeEmpty = 24;  // 2
+constexpr int kBarSFull = 26;
+constexpr int kBarSEmpty = 27;     // one arrival per softmax warp
+constexpr int kBarPFull = 28;      // one arrival per softmax warp
+constexpr int kBarPEmpty = 29;
+constexpr int kBarOReady = 30;     // 2: per tile parity (the rescale loop may run a tile ahead)
+constexpr int kBarPvDone = 32;
+constexpr int kBarQReady = 33;     // one arrival per softmax warp
+constexpr int kBarAlphaFull = 34;  // 2: per tile parity, one arrival per lane quadrant
+constexpr int kBarDrain = 36;
+constexpr int kNumBars = 37;
 
 struct Scratch {
-  uint64_t bars[32];
+  uint64_t bars[40];
   uint32_t tmem_base;
   int abort;
   int pad[2];
-  float warp_max[4][4][16];  // per softmax group, per warp, per column; reused for row sums
-  float m_run[64];           // max used per column (log2 units)
-  float alpha[2][64];        // per tile parity: rescale factor per column
-  uint32_t changed[2][4];    // per tile parity, per softmax group: columns whose max moved
-  float c_head[64];          // per column: softmax_scale * kv_scale * log2(e) * 2^-e
-  float inv_l[64];           // per column: kv_scale / l  (0 when l == 0)
-  uint8_t qcol[64];          // per column: its query position q
+  float red[4][64];          // per token slice, per query row: amax, tile max, row sums
+  float m_run[64];           // max used per query row (log2 units), for the epilogue/merge
+  float inv_l[64];           // per query row: kv_scale / l (0 when l == 0), or raw l when cut
+  float alpha[2][64];        // per tile parity: rescale factor per query row
+  uint32_t changed[2][4];    // per tile parity, per lane quadrant: rows whose max moved
 };
 static_assert(kOffScratch + sizeof(Scratch) <= kSmemBytes, "shared memory overflow");
+static_assert(kNumBars <= 40, "barrier array");
 
 // 64-byte swizzle of a 64-byte-row layout: 16-byte unit u of row r lives at
 // unit u ^ ((r >> 1) & 3).  Matches the TMA 64B swizzle and the UMMA SW64
 // canonical layout when the atom base is 512-byte aligned.
 __device__ __forceinline__ uint32_t sw64(uint32_t row, uint32_t byte_in_row) {
   return row * 64u + ((((byte_in_row >> 4) ^ ((row >> 1) & 3u)) << 4) | (byte_in_row & 15u));
+}
+// 128-byte swizzle of a 128-byte-row layout: unit u of row r at u ^ (r & 7)
+// (UMMA SW128 canonical layout for a 1024-byte-aligned atom base).
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t byte_in_row) {
+  return row * 128u + ((((byte_in_row >> 4) ^ (row & 7u)) << 4) | (byte_in_row & 15u));
 }
 
 __device__ __forceinline__ void set_error(int32_t* err, int bit) {
@@ -139,24 +153,37 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t bytes) {
   return base + (uint64_t)(bytes >> 4);
 }
 
-// Split 8 fp32 values into two E4M3 terms each: hi = x rounded to 4
-// significant bits (round half away from zero on the bit pattern; an exact
-// E4M3 value for |x| in the normal range), lo = E4M3(x - hi).  Result bytes
-// are in element order.
-__device__ __forceinline__ void split8(const float* x, uint2& hi, uint2& lo) {
-  uint32_t h[4], l[4];
+// x rounded to 4 significant bits (round half away from zero on the bit
+// pattern): an exact E4M3 value for |x| in the normal range.
+__device__ __forceinline__ float hi4(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x80000u) & 0xFFF00000u);
+}
+
+// Split 16 fp32 values into two E4M3 terms each: hi = hi4(x), lo = E4M3(x -
+// hi).  Result bytes are in element order (16 bytes per term).
+__device__ __forceinline__ void split16(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[8], l[8];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < 8; ++k) {
     const float a = x[2 * k], b = x[2 * k + 1];
-    const float ha = __uint_as_float((__float_as_uint(a) + 0x80000u) & 0xFFF00000u);
-    const float hb = __uint_as_float((__float_as_uint(b) + 0x80000u) & 0xFFF00000u);
+    const float ha = hi4(a), hb = hi4(b);
     h[k] = cvt_e4m3x2(ha, hb);
     l[k] = cvt_e4m3x2(a - ha, b - hb);
   }
-  hi.x = h[0] | (h[1] << 16);
-  hi.y = h[2] | (h[3] << 16);
-  lo.x = l[0] | (l[1] << 16);
-  lo.y = l[2] | (l[3] << 16);
+  hi = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+  lo = make_uint4(l[0] | (l[1] << 16), l[2] | (l[3] << 16), l[4] | (l[5] << 16), l[6] | (l[7] << 16));
+}
+
+// One term (hi or lo) of 8 fp32 values as E4M3 codes, element order.
+__device__ __forceinline__ uint2 term8(const float* x, bool lo) {
+  uint32_t c[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float a = x[2 * k], b = x[2 * k + 1];
+    const float ha = hi4(a), hb = hi4(b);
+    c[k] = lo ? cvt_e4m3x2(a - ha, b - hb) : cvt_e4m3x2(ha, hb);
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 // Merge of the P CTAs (one cluster) that share a split, each having staged
@@ -296,7 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int p1 = min(p0 + cpages, n_pages);
   const int r0 = g * kRows;
   const int rows_valid = min(kRows, QH - r0);
-  const int q_min = r0 / args.H;
   const int q_max = (r0 + rows_valid - 1) / args.H;
   const int vis_base = L - args.q_len + 1;  // visible length of q = 0
   const int t0s = p0 * 64;                         // the split's tokens [t0s, t1s)
@@ -321,7 +347,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pg0 = p0 + 2 * tile0;      // block-table index of the run's first page
   const int t0 = t0s + tile0 * kTile;
   const int t1 = min(t1s, t0 + T * kTile);
-  const int t_all = min(t1, vis_base + q_min);  // every column sees every token < t_all
 
   // ---------------------------------------------------------------- setup
   if ((smem_u32(smem) & 1023u) != 0) {  // same for every CTA of the grid
@@ -340,28 +365,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     for (int i = 0; i < kRingPairs; ++i) {
-      mbar_init(&sc.bars[kBarNopeFull + i], 1);
-      mbar_init(&sc.bars[kBarNopeEmpty + i], 1);
+      mbar_init(&sc.bars[kBarFull + i], 1);
+      mbar_init(&sc.bars[kBarEmpty + i], 1);
     }
-    mbar_init(&sc.bars[kBarRopeFull], 1);
-    mbar_init(&sc.bars[kBarRopeEmpty], 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sc.bars[kBarSFull + i], 1);
-      mbar_init(&sc.bars[kBarSEmpty + i], kSoftThreads);
+    for (int i = 0; i < kRopeSlots; ++i) {
+      mbar_init(&sc.bars[kBarRopeFull + i], 1);
+      mbar_init(&sc.bars[kBarRopeEmpty + i], 1);
     }
-    mbar_init(&sc.bars[kBarPFull], kSoftThreads);
+    mbar_init(&sc.bars[kBarSFull], 1);
+    mbar_init(&sc.bars[kBarSEmpty], kSoftWarps);
+    mbar_init(&sc.bars[kBarPFull], kSoftWarps);
     mbar_init(&sc.bars[kBarPEmpty], 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarOReady + i], 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarOReady + i], 4);
     mbar_init(&sc.bars[kBarPvDone], 1);
-    mbar_init(&sc.bars[kBarQReady], 4 * kSoftGroups);
-    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarAlphaFull + i], kSoftGroups);
+    mbar_init(&sc.bars[kBarQReady], kSoftWarps);
+    for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarAlphaFull + i], 4);
     mbar_init(&sc.bars[kBarDrain], 1);
     sc.abort = 0;
     fence_barrier_init();
-  }
-  if (tid < 64) {
-    sc.m_run[tid] = -INFINITY;
-    sc.qcol[tid] = (uint8_t)min((r0 + tid) / args.H, 255);
   }
   if (warp == 1) {
     tmem_alloc(&sc.tmem_base, 512);
@@ -377,7 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     // The whole warp runs this loop with warp-uniform values; one elected
-    // lane issues each TMA instruction and barrier arrival.
+    // lane issues each TMA instruction and barrier arrival.  Latent pair j of
+    // tile i is load number u = 4 i + j and goes to ring slot u % 11; the
+    // RoPE chunk of tile i goes to slot i % 2 of its own ring.
     if (lane == 0) prefetch_tensormap(&kv_map);
     __syncwarp();
     const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
@@ -394,14 +417,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (want_b && pb >= 0 && (int64_t)pb < args.num_pages)
         bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pb * kPageBytes, kPageBytes);
     };
-    if (T > 2) prefetch_tile(2);
-    int last_nope_parity[kRingPairs];
+    constexpr int kAhead = 2;  // tiles prefetched into L2 ahead of the one being loaded
+    for (int i = 1; i < min(T, kAhead); ++i) prefetch_tile(i);
+    int last_parity[kRingPairs];
     bool armed[kRingPairs];
     for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
-    int rope_armed_tiles = 0;
+    int rope_last[kRopeSlots] = {-1, -1};
     bool ok = true;
+    int u = 0;  // load number of the next latent pair
     for (int i = 0; i < T && ok; ++i) {
-      if (i + 3 < T) prefetch_tile(i + 3);
+      if (i + kAhead < T) prefetch_tile(i + kAhead);
       const int tok0 = t0 + i * kTile;
       const int pa = bt[pg0 + 2 * i];
       const bool want_b = tok0 + 64 < t1;
@@ -410,19 +435,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool lb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
       if (lane == 0 && (!la || (want_b && !lb))) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
       const uint32_t bytes_chunk = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
-      for (int j = 0; j < 4; ++j) {
-        const int slot = (i & 1) * 4 + j;
-        if (i >= 2) {
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(&bars[kBarNopeEmpty + slot], ((i - 2) >> 1) & 1, abort_flag));
+      for (int j = 0; j < 4; ++j, ++u) {
+        const int slot = u % kRingPairs;
+        const int use = u / kRingPairs;  // how many times the slot was filled before
+        if (use >= 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarEmpty + slot], (use - 1) & 1, abort_flag));
           if (!ok) break;
         }
-        uint64_t* full = &bars[kBarNopeFull + slot];
+        uint64_t* full = &bars[kBarFull + slot];
         if (args.inject_stall && i == 0 && j == 0 && blockIdx.x == 0)
           continue;  // test hook: this slot is never armed, so its waits run out
         mbar_arrive_expect_tx_elect(full, 2 * bytes_chunk);
         armed[slot] = true;
-        last_nope_parity[slot] = (i >> 1) & 1;
+        last_parity[slot] = use & 1;
         uint8_t* dst = smem + kOffRing + slot * kPair;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -432,40 +457,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarRopeEmpty], (i - 1) & 1, abort_flag));
+      const int rs = i % kRopeSlots;
+      if (i >= kRopeSlots) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars[kBarRopeEmpty + rs], ((i / kRopeSlots) - 1) & 1, abort_flag));
         if (!ok) break;
       }
-      uint64_t* rfull = &bars[kBarRopeFull];
+      uint64_t* rfull = &bars[kBarRopeFull + rs];
       mbar_arrive_expect_tx_elect(rfull, bytes_chunk);
-      rope_armed_tiles = i + 1;
-      if (la) tma_load_3d_elect(smem + kOffRope, &kv_map, rfull, 512, 0, pa);
-      if (lb) tma_load_3d_elect(smem + kOffRope + 4096, &kv_map, rfull, 512, 0, pb);
+      rope_last[rs] = i;
+      uint8_t* rdst = smem + kOffRope + rs * kChunk;
+      if (la) tma_load_3d_elect(rdst, &kv_map, rfull, 512, 0, pa);
+      if (lb) tma_load_3d_elect(rdst + 4096, &kv_map, rfull, 512, 0, pb);
     }
     // drain: every armed transaction has landed before the CTA may exit
     const uint64_t t_start = globaltimer_ns();
     for (int i = 0; i < kRingPairs; ++i)
       if (armed[i])
-        while (!mbar_try_wait(&bars[kBarNopeFull + i], last_nope_parity[i]) &&
+        while (!mbar_try_wait(&bars[kBarFull + i], last_parity[i]) &&
                globaltimer_ns() - t_start < kWaitLimitNs) {
         }
-    if (rope_armed_tiles > 0)
-      while (!mbar_try_wait(&bars[kBarRopeFull], (rope_armed_tiles - 1) & 1) &&
-             globaltimer_ns() - t_start < kWaitLimitNs) {
-      }
+    for (int rs = 0; rs < kRopeSlots; ++rs)
+      if (rope_last[rs] >= 0)
+        while (!mbar_try_wait(&bars[kBarRopeFull + rs], (rope_last[rs] / kRopeSlots) & 1) &&
+               globaltimer_ns() - t_start < kWaitLimitNs) {
+        }
   } else if (warp == 1) {
     // ============================================================ UMMA issuer
     // Warp-uniform scheduler; one elected lane issues each MMA and commit.
-    const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, 128, 128);  // E4M3 K-major x K-major, N=128
-    const uint32_t idesc_pv = instr_desc(0, 0, 1, 1, 128, 64);   // MN-major x MN-major, N=64
-    // K-major SW64 (8-row groups 512 B apart) and MN-major SW64 (64-element
-    // atoms 8 KiB apart, 8-row groups 512 B apart) descriptor bases
+    const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, 128, 128);  // E4M3, A K-major (TMEM or smem), B K-major, N=128
+    const uint32_t idesc_pv = instr_desc(0, 0, 1, 0, 128, 64);   // A MN-major, B K-major, N=64
+    // K-major SW64 (8-row groups 512 B apart), MN-major SW64 (64-element
+    // atoms 8 KiB apart, 8-row groups 512 B apart), K-major SW128 (8-row
+    // groups 1 KiB apart) descriptor bases
     const uint64_t dRingK = smem_desc(smem_u32(smem + kOffRing), 16, 512, 4);
     const uint64_t dRope = smem_desc(smem_u32(smem + kOffRope), 16, 512, 4);
-    const uint64_t dQ = smem_desc(smem_u32(smem + kOffQ), 16, 512, 4);
+    const uint64_t dQr = smem_desc(smem_u32(smem + kOffQr), 16, 512, 4);
     const uint64_t dRingMN = smem_desc(smem_u32(smem + kOffRing), kChunk, 512, 4);
-    const uint64_t dPhi = smem_desc(smem_u32(smem + kOffPhi), kChunk, 512, 4);
-    const uint64_t dPlo = smem_desc(smem_u32(smem + kOffPlo), kChunk, 512, 4);
+    const uint64_t dPhi = smem_desc(smem_u32(smem + kOffPhi), 16, 1024, 2);
+    const uint64_t dPlo = smem_desc(smem_u32(smem + kOffPlo), 16, 1024, 2);
+    const uint32_t d_s = tmem + kTmemS;
     auto ready = [&](int bar, int parity) {
       return __any_sync(0xffffffffu, mbar_test_wait(&bars[bar], parity));
     };
@@ -477,64 +508,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t idle_spins = 0;
     while (ok && np < T) {
       bool progress = false;
-      // ---------------- S^T(nq) = K(nq) . [Q_hi ; Q_lo]^T, one 128-dim pair at a time
-      if (nq < T) {
-        const int sb = nq & 1;
-        const uint32_t d_s = tmem + sb * 128;
-        if (!s_free) {
-          s_free = nq < 2 || ready(kBarSEmpty + sb, ((nq - 2) >> 1) & 1);
-          if (s_free) tc_fence_after();
-        }
-        while (s_free && qpair < 4 && ready(kBarNopeFull + (nq & 1) * 4 + qpair, (nq >> 1) & 1)) {
-          tc_fence_after();
-          const uint32_t a_off = ((nq & 1) * 4 + qpair) * kPair;
-          const uint32_t b_off = 2 * qpair * kChunk;
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              umma_f8_elect(d_s, desc_at(dRingK, a_off + cc * kChunk + kk * 32),
-                            desc_at(dQ, b_off + cc * kChunk + kk * 32), idesc_qk,
-                            (qpair | cc | kk) != 0 ? 1u : 0u);
-          ++qpair;
-          progress = true;
-        }
-        if (s_free && qpair == 4 && ready(kBarRopeFull, nq & 1)) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            umma_f8_elect(d_s, desc_at(dRope, kk * 32), desc_at(dQ, 8 * kChunk + kk * 32),
-                          idesc_qk, 1u);
-          umma_commit_elect(&bars[kBarSFull + sb]);
-          umma_commit_elect(&bars[kBarRopeEmpty]);
-          ++nq;
-          qpair = 0;
-          s_free = false;
-          progress = true;
-        }
-      }
-      // ---------------- O^T += V(np)^T . (P_hi + P_lo)
+      // ---------------- O^T += V(np)^T . (P_hi + P_lo), before any further QK
       if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady + (np & 1), (np >> 1) & 1)) {
         tc_fence_after();
-        const uint32_t slot0 = (np & 1) * 4 * kPair;
         // block by block, so each latent pair can be refilled as soon as its
         // block is done
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+          const int slot = (4 * np + j) % kRingPairs;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-            for (int hl = 0; hl < 2; ++hl)
-              umma_f8_elect(tmem + 256 + 64 * j, desc_at(dRingMN, slot0 + j * kPair + kk * 2048),
-                            desc_at(hl ? dPlo : dPhi, kk * 2048), idesc_pv,
-                            (np > 0 || kk > 0 || hl > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = desc_at(dRingMN, slot * kPair + kk * 2048);
+            umma_f8_fill_elect(tmem + kTmemO + 64 * j, a, desc_at(dPhi, kk * 32), idesc_pv,
+                               (np > 0 || kk > 0) ? 1u : 0u);
+            umma_f8_lastuse_elect(tmem + kTmemO + 64 * j, a, desc_at(dPlo, kk * 32), idesc_pv, 1u);
+          }
           // latent pair j of this tile is free once its block's MMAs complete
-          umma_commit_elect(&bars[kBarNopeEmpty + (np & 1) * 4 + j]);
+          umma_commit_elect(&bars[kBarEmpty + slot]);
         }
         umma_commit_elect(&bars[kBarPEmpty]);
         umma_commit_elect(&bars[kBarPvDone]);
         ++np;
         progress = true;
+      }
+      // ---------------- S'(nq) = Q' . K(nq)^T, one 128-dim pair at a time
+      if (nq < T) {
+        if (!s_free) {
+          s_free = nq < 1 || ready(kBarSEmpty, (nq - 1) & 1);
+          if (s_free) tc_fence_after();
+        }
+        while (s_free && qpair < 4 &&
+               ready(kBarFull + (4 * nq + qpair) % kRingPairs, ((4 * nq + qpair) / kRingPairs) & 1)) {
+          tc_fence_after();
+          const uint32_t b_off = ((4 * nq + qpair) % kRingPairs) * kPair;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int ks = 4 * qpair + 2 * cc + kk;  // K step of 32 latent dims
+              umma_f8_ts_elect(d_s, tmem + kTmemQ + 8 * ks, desc_at(dRingK, b_off + cc * kChunk + kk * 32),
+                               idesc_qk, ks != 0 ? 1u : 0u);
+            }
+          ++qpair;
+          progress = true;
+        }
+        if (s_free && qpair == 4 && ready(kBarRopeFull + nq % kRopeSlots, (nq / kRopeSlots) & 1)) {
+          tc_fence_after();
+          const uint32_t r_off = (nq % kRopeSlots) * kChunk;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            umma_f8_elect(d_s, desc_at(dQr, kk * 32), desc_at(dRope, r_off + kk * 32), idesc_qk, 1u);
+          umma_commit_elect(&bars[kBarSFull]);
+          umma_commit_elect(&bars[kBarRopeEmpty + nq % kRopeSlots]);
+          ++nq;
+          qpair = 0;
+          s_free = false;
+          progress = true;
+        }
       }
       if (progress) {
         idle_spins = 0;
@@ -554,211 +584,211 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t t_start = globaltimer_ns();
     while (!mbar_try_wait(&bars[kBarDrain], 0) && globaltimer_ns() - t_start < kWaitLimitNs) {
     }
-  } else if (warp >= 4 && warp < 4 + 4 * kSoftGroups) {
+  } else if (warp >= 4 && warp < 4 + kSoftWarps) {
     // ============================================================ Q split + softmax
-    const int wg = (warp - 4) >> 2;  // softmax group: query columns 16*wg .. 16*wg+15
-    const int wq = warp & 3;         // TMEM lane quadrant
+    const int qd = warp & 3;           // TMEM lane quadrant
+    const int c = (warp - 4) >> 2;     // token slice: tokens 32c .. 32c+31 of a tile
+    const int part = lane >> 4;        // 0: hi term, 1: lo term
+    const int n = 16 * qd + (lane & 15);  // query row of this thread
+    const bool valid = n < rows_valid;
+    const int bar_id = 1 + qd;         // the four warps of this quadrant
+    float c_head;                      // softmax_scale * kv_scale * log2(e) * 2^-e
     {
-      // ---- Q -> [Q_hi ; Q_lo] in K-major SW64 chunks, per-row power-of-two scale
-      const int pw = warp - 4;  // rows pw, pw + 16, ...
-      for (int n = pw; n < kRows; n += 4 * kSoftGroups) {
-        const bool valid = n < rows_valid;
-        const uint16_t* qn = args.q_nope + (row_base + n) * 512;
-        const uint16_t* qr = args.q_rope + (row_base + n) * 64;
-        uint4 v[3];
-        const int nch = lane < 8 ? 3 : 2;
-        const int dim0[3] = {lane * 8, 256 + lane * 8, 512 + lane * 8};
-        v[0] = valid ? *reinterpret_cast<const uint4*>(qn + lane * 8) : make_uint4(0, 0, 0, 0);
-        v[1] = valid ? *reinterpret_cast<const uint4*>(qn + 256 + lane * 8) : make_uint4(0, 0, 0, 0);
-        v[2] = (valid && lane < 8) ? *reinterpret_cast<const uint4*>(qr + lane * 8)
-                                   : make_uint4(0, 0, 0, 0);
-        uint32_t amax_bits = 0;
-        for (int c = 0; c < nch; ++c) {
-          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+      // ---- Q -> Q' = [Q_hi ; Q_lo] with a power-of-two scale per query row:
+      // this thread converts latent dims [128c, 128c+128) and RoPE dims
+      // [16c, 16c+16) of row n, term `part`; the latent bytes go to TMEM lane
+      // 32 qd + lane, the RoPE bytes to shared memory row 32 qd + lane.  The
+      // row's amax is taken over all 576 dims (the four slices of the row).
+      const uint16_t* qn = args.q_nope + (row_base + n) * 512 + 128 * c;
+      const uint16_t* qr = args.q_rope + (row_base + n) * 64 + 16 * c;
+      auto load8 = [&](int k) -> uint4 {  // dims 8k .. 8k+7 of the slice (k >= 16: RoPE)
+        if (!valid) return make_uint4(0, 0, 0, 0);
+        return k < 16 ? *reinterpret_cast<const uint4*>(qn + 8 * k)
+                      : *reinterpret_cast<const uint4*>(qr + 8 * (k - 16));
+      };
+      uint32_t amax_bits = 0;
+#pragma unroll 6
+      for (int k = 0; k < 18; ++k) {
+        const uint4 v = load8(k);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            amax_bits = max(amax_bits, (w[k] << 16) & 0x7FFFFFFFu);
-            amax_bits = max(amax_bits, w[k] & 0x7FFF0000u);
+        for (int e = 0; e < 4; ++e) {
+          amax_bits = max(amax_bits, (w[e] << 16) & 0x7FFFFFFFu);
+          amax_bits = max(amax_bits, w[e] & 0x7FFF0000u);
+        }
+      }
+      if (part == 0) sc.red[c][n] = __uint_as_float(amax_bits);
+      named_bar_sync(bar_id, 128);
+      const float amax = fmaxf(fmaxf(sc.red[0][n], sc.red[1][n]), fmaxf(sc.red[2][n], sc.red[3][n]));
+      int e = 0;
+      if (amax > 0.0f && __float_as_uint(amax) < 0x7F800000u) {
+        int E;
+        frexpf(amax, &E);    // amax in [2^(E-1), 2^E)
+        e = min(max(8 - E, -126), 126);  // amax * 2^e in [128, 256)
+      }
+      c_head = valid ? args.qk_scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23) : 0.0f;
+      const float sc_up = __uint_as_float((uint32_t)(127 + e) << 23);
+      auto term_of = [&](int k) -> uint2 {  // this thread's term of dims 8k .. 8k+7
+        const uint4 v = load8(k);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float x[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          x[2 * e2] = __uint_as_float(w[e2] << 16) * sc_up;
+          x[2 * e2 + 1] = __uint_as_float(w[e2] & 0xFFFF0000u) * sc_up;
+        }
+        return term8(x, part != 0);
+      };
+      const uint32_t t_q = tmem + ((uint32_t)(32 * qd) << 16) + kTmemQ + 32 * c;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // 64 latent dims = 16 TMEM columns at a time
+        float cols[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint2 t8 = term_of(8 * h + k);
+          cols[2 * k] = __uint_as_float(t8.x);
+          cols[2 * k + 1] = __uint_as_float(t8.y);
+        }
+        tmem_st16(t_q + 16 * h, cols);
+      }
+#pragma unroll
+      for (int k = 16; k < 18; ++k)
+        *reinterpret_cast<uint2*>(smem + kOffQr + sw64(32 * qd + lane, 16 * c + 8 * (k - 16))) = term_of(k);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarQReady]);
+    }
+
+    // ---- softmax over S': this thread ends up with the scores of row n for
+    // the 16 tokens 32c + 16 part .. +15 of each tile
+    const int q_of_row = (r0 + n) / args.H;
+    const int lim = valid ? min(t1, vis_base + q_of_row) : t0;  // tokens >= lim are invisible
+    const uint32_t t_s = tmem + ((uint32_t)(32 * qd) << 16) + kTmemS + 32 * c;
+    const int tid_s = tid - 128;       // 0..511
+    float m_run = -INFINITY;           // max used for row n (log2 units)
+    float l_run = 0.0f;                // this thread's share of row n's sum
+    bool bad = false;
+    for (int i = 0; i < T; ++i) {
+      const int tok_base = t0 + i * kTile + 32 * c + 16 * part;
+      bad |= !mbar_wait(&bars[kBarSFull], i & 1, abort_flag);
+      tc_fence_after();
+      float sv[16];
+      {
+        uint32_t r[32];
+        tmem_ld32_nowait(t_s, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarSEmpty]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float keep = __uint_as_float(part ? r[16 + j] : r[j]);
+          const float give = __uint_as_float(part ? r[j] : r[16 + j]);
+          sv[j] = (keep + __shfl_xor_sync(0xffffffffu, give, 16)) * c_head;
+        }
+      }
+      // visibility mask (split end, causal limit of the row, sequence end)
+      if (tok_base + 16 > lim) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (tok_base + j >= lim) sv[j] = -INFINITY;
+      }
+      // does any score exceed the used max by more than the lazy threshold?
+      bool exceed = false;
+      const float thr = m_run + kLazy;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) exceed |= sv[j] > thr;
+      float alpha = 1.0f;
+      bool moved = false;
+      // One vote per quadrant and tile; its result is the same for all 128
+      // threads, so they take the same barriers.  After a failed wait (bad)
+      // a thread keeps looping: its waits return at once, the results are
+      // discarded, and no thread is left at a named barrier.
+      if (named_bar_or(bar_id, 128, exceed || bad)) {
+        // some row of this quadrant may move: tile max per row over the 128 tokens
+        float tm = sv[0];
+#pragma unroll
+        for (int j = 1; j < 16; ++j) tm = fmaxf(tm, sv[j]);
+        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+        if (part == 0) sc.red[c][n] = tm;
+        named_bar_sync(bar_id, 128);
+        tm = fmaxf(fmaxf(sc.red[0][n], sc.red[1][n]), fmaxf(sc.red[2][n], sc.red[3][n]));
+        moved = tm > thr;
+        if (moved) {
+          alpha = m_run == -INFINITY ? 0.0f : ex2_approx(m_run - tm);
+          m_run = tm;
+        }
+      }
+      // the rescale warps learn, per tile, which rows moved and by how much
+      if (c == 0) {
+        const uint32_t mask = __ballot_sync(0xffffffffu, moved && part == 0);
+        if (part == 0) sc.alpha[i & 1][n] = alpha;
+        if (lane == 0) sc.changed[i & 1][qd] = mask & 0xFFFFu;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
+      }
+      // weights carry a 2^7 factor: p' = 2^(s - m + 7) <= 2^8.75
+      float pv[16];
+      float psum = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        pv[j] = (sv[j] == -INFINITY) ? 0.0f : ex2_approx(sv[j] - m_run + kPShift);
+        psum += pv[j];
+      }
+      l_run = fmaf(l_run, alpha, psum);
+      uint4 phi, plo;
+      split16(pv, phi, plo);
+      // P buffer (and the V rows cleared below) free: PV of the previous tile done
+      if (i >= 1) bad |= !mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
+      const uint32_t p_off = sw128(n, 32 * c + 16 * part);
+      *reinterpret_cast<uint4*>(smem + kOffPhi + p_off) = phi;
+      *reinterpret_cast<uint4*>(smem + kOffPlo + p_off) = plo;
+      if (t0 + i * kTile + kTile > t1) {
+        // token rows past the visible range: clear their V bytes so that
+        // 0 * garbage cannot be NaN (thread: token row tid_s & 127, pair tid_s >> 7)
+        const int r = tid_s & 127;
+        if (t0 + i * kTile + r >= t1) {
+          const int slot = (4 * i + (tid_s >> 7)) % kRingPairs;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + slot * kPair + cc * kChunk + r * 64);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) row[k] = make_uint4(0, 0, 0, 0);
           }
         }
-        amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
-        const float amax = __uint_as_float(amax_bits);
-        int e = 0;
-        if (amax > 0.0f && amax_bits < 0x7F800000u) {
-          int E;
-          frexpf(amax, &E);    // amax in [2^(E-1), 2^E)
-          e = min(max(8 - E, -126), 126);  // amax * 2^e in [128, 256)
-        }
-        const float sc_up = __uint_as_float((uint32_t)(127 + e) << 23);
-        for (int c = 0; c < nch; ++c) {
-          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-          float x[8];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            x[2 * k] = __uint_as_float(w[k] << 16) * sc_up;
-            x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u) * sc_up;
-          }
-          uint2 hi, lo;
-          split8(x, hi, lo);
-          const int chunk = dim0[c] >> 6;
-          const uint32_t bo = dim0[c] & 63;
-          uint8_t* base = smem + kOffQ + chunk * kChunk;
-          *reinterpret_cast<uint2*>(base + sw64(n, bo)) = hi;
-          *reinterpret_cast<uint2*>(base + sw64(64 + n, bo)) = lo;
-        }
-        if (lane == 0)
-          sc.c_head[n] = valid ? args.qk_scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23)
-                               : 0.0f;
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarQReady]);
-      named_bar_sync(7, kSoftThreads);  // c_head visible to every softmax group
+      if (lane == 0) mbar_arrive(&bars[kBarPFull]);
     }
-
-    // ---- softmax over S^T: thread = token row r of the tile, 16 query columns
-    const int r = wq * 32 + lane;
-    const int col0 = wg * kCols;
-    const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-    const float4* c4 = reinterpret_cast<const float4*>(sc.c_head + col0);
-    float l_part[kCols];
-#pragma unroll
-    for (int j = 0; j < kCols; ++j) l_part[j] = 0.0f;
-    const int bar_id = 1 + wg;
-    bool ok = true;
-    bool bad = false;
-    for (int i = 0; i < T; ++i) {
-      const int sb = i & 1;
-      const int tok = t0 + i * kTile + r;
-      bad |= !mbar_wait(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag);
-      tc_fence_after();
-      float sv[kCols];
-      {
-        float hi[kCols], lo[kCols];
-        const uint32_t ts = t_lane + sb * 128 + col0;
-        tmem_ld16x2(ts, ts + 64, hi, lo);
-#pragma unroll
-        for (int j4 = 0; j4 < kCols / 4; ++j4) {
-          const float4 c = c4[j4];
-          sv[4 * j4 + 0] = (hi[4 * j4 + 0] + lo[4 * j4 + 0]) * c.x;
-          sv[4 * j4 + 1] = (hi[4 * j4 + 1] + lo[4 * j4 + 1]) * c.y;
-          sv[4 * j4 + 2] = (hi[4 * j4 + 2] + lo[4 * j4 + 2]) * c.z;
-          sv[4 * j4 + 3] = (hi[4 * j4 + 3] + lo[4 * j4 + 3]) * c.w;
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[kBarSEmpty + sb]);
-      // visibility mask (split end, causal limit per column, sequence end)
-      if (t0 + i * kTile + kTile > t_all) {
-        const int qq = tok - vis_base;  // token invisible to columns whose q <= qq
-#pragma unroll
-        for (int j = 0; j < kCols; ++j)
-          if (tok >= t1 || (qq >= 0 && (int)sc.qcol[col0 + j] <= qq)) sv[j] = -INFINITY;
-      }
-      // per-column tile max: warp redux, then across the 4 warps
-      float mine = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < kCols; ++j) {
-        const float wm = warp_max_f32(sv[j]);
-        mine = (lane == j) ? wm : mine;
-      }
-      if (lane < kCols) sc.warp_max[wg][wq][lane] = mine;
-      if (named_bar_or(bar_id, 128, bad || *abort_flag != 0)) {
-        ok = false;
-        break;
-      }
-      if (wq == 0) {
-        const int n = col0 + lane;
-        bool moved = false;
-        if (lane < kCols) {
-          const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
-                                 fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
-          const float m_old = sc.m_run[n];
-          moved = tm > m_old + kLazy;
-          const float m_new = moved ? tm : m_old;
-          const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
-          sc.m_run[n] = m_new;
-          sc.alpha[i & 1][n] = a;
-        }
-        const uint32_t mask = __ballot_sync(0xffffffffu, moved);
-        if (lane == 0) sc.changed[i & 1][wg] = mask;
-      }
-      named_bar_sync(bar_id, 128);
-      if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
-      const float4* m4 = reinterpret_cast<const float4*>(sc.m_run + col0);
-      const float4* a4 = reinterpret_cast<const float4*>(sc.alpha[i & 1] + col0);
-      uint2 phi[kCols / 8], plo[kCols / 8];
-#pragma unroll
-      for (int q8 = 0; q8 < kCols / 8; ++q8) {
-        const float4 ma = m4[2 * q8], mb = m4[2 * q8 + 1];
-        const float4 aa = a4[2 * q8], ab = a4[2 * q8 + 1];
-        const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-        const float al[8] = {aa.x, aa.y, aa.z, aa.w, ab.x, ab.y, ab.z, ab.w};
-        float pv[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int j = 8 * q8 + k;
-          // weights carry a 2^7 factor: p' = 2^(s - m + 7) <= 2^8.75
-          pv[k] = (sv[j] == -INFINITY) ? 0.0f : ex2_approx(sv[j] - mm[k] + kPShift);
-          l_part[j] = fmaf(l_part[j], al[k], pv[k]);
-        }
-        split8(pv, phi[q8], plo[q8]);
-      }
-      // P buffer (and the V rows cleared below) free: PV of the previous tile done
-      if (i >= 1) bad |= !mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
-      *reinterpret_cast<uint4*>(smem + kOffPhi + sw64(r, col0)) =
-          make_uint4(phi[0].x, phi[0].y, phi[1].x, phi[1].y);
-      *reinterpret_cast<uint4*>(smem + kOffPlo + sw64(r, col0)) =
-          make_uint4(plo[0].x, plo[0].y, plo[1].x, plo[1].y);
-      if (tok >= t1) {
-        // rows past the visible range: clear their V bytes so 0 * garbage cannot be NaN
-        // (softmax group g clears latent pair g)
-        const int pair = (i & 1) * 4 + wg;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + pair * kPair + cc * kChunk + r * 64);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) row[u] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kBarPFull]);
-    }
-    // ---- row sums: reduce l_part over the 128 token rows of this group
+    // ---- row sums: reduce l over the 8 threads of row n, in a fixed order
     {
-      float mine = 0.0f;
-#pragma unroll
-      for (int j = 0; j < kCols; ++j) {
-        float v = l_part[j];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        mine = (lane == j) ? v : mine;
-      }
-      named_bar_sync(bar_id, 128);  // warp_max no longer read
-      if (lane < kCols) sc.warp_max[wg][wq][lane] = mine;
+      const float l2 = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      named_bar_sync(bar_id, 128);  // red no longer read
+      if (part == 0) sc.red[c][n] = l2;
       named_bar_sync(bar_id, 128);
-      if (wq == 0 && lane < kCols) {
-        const int n = col0 + lane;
-        const float l = (sc.warp_max[wg][0][lane] + sc.warp_max[wg][1][lane]) +
-                        (sc.warp_max[wg][2][lane] + sc.warp_max[wg][3][lane]);
-        const bool nonempty = ok && l > 0.0f;
+      if (c == 0 && part == 0) {
+        const float l = (sc.red[0][n] + sc.red[1][n]) + (sc.red[2][n] + sc.red[3][n]);
+        const bool nonempty = !bad && l > 0.0f;
+        sc.m_run[n] = m_run;
         if (npieces == 1) {
           sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
-          if (n < rows_valid)
+          if (valid)
             args.part_lse[(row_base + n) * args.max_splits + s] =
-                nonempty ? (sc.m_run[n] - kPShift + log2f(l)) * 0.69314718055994530942f
-                         : -INFINITY;
+                nonempty ? (m_run - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
         } else {
           sc.inv_l[n] = nonempty ? l : 0.0f;  // raw row sum, merged across the cluster
         }
       }
     }
     named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
-  } else if (warp >= 4 + 4 * kSoftGroups) {
+  } else if (warp >= 4 + kSoftWarps) {
     // ============================================================ O^T rescale between tiles
     // The O-ready barriers are per tile parity because this loop may run one
-    // tile ahead of the PV issue, but never two: tile i + 2 needs the ring
-    // slots that PV(i) frees, and so its max and alpha.
+    // tile ahead of the PV issue, but never two: the softmax of tile i + 2
+    // needs the P buffer that PV(i) frees, and so its max and alpha.
     const int wq = warp & 3;            // thread = latent dim wq * 32 + lane of a block
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     bool ok = true;
@@ -771,31 +801,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ch0 = i >= 1 ? sc.changed[i & 1][0] : 0u, ch1 = i >= 1 ? sc.changed[i & 1][1] : 0u;
       const uint32_t ch2 = i >= 1 ? sc.changed[i & 1][2] : 0u, ch3 = i >= 1 ? sc.changed[i & 1][3] : 0u;
       if ((ch0 | ch1 | ch2 | ch3) != 0) {
-        // some column's max moved: O^T is rescaled once PV of the previous tile is done
+        // some row's max moved: O^T is rescaled once PV of the previous tile is done
         if (wq == 0 && lane == 0) mbar_wait(&bars[kBarPvDone], (i - 1) & 1, abort_flag);
         named_bar_sync(5, 128);
         tc_fence_after();
 #pragma unroll 1
-        for (int grp = 0; grp < 4; ++grp) {  // grp = softmax group = 16 columns
+        for (int grp = 0; grp < 4; ++grp) {  // grp = lane quadrant = 16 query rows
           const uint32_t bits = grp == 0 ? ch0 : grp == 1 ? ch1 : grp == 2 ? ch2 : ch3;
           if (bits == 0) continue;
           float a[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) a[c] = sc.alpha[i & 1][grp * 16 + c];
+          for (int k = 0; k < 16; ++k) a[k] = sc.alpha[i & 1][grp * 16 + k];
 #pragma unroll 1
           for (int j = 0; j < 4; ++j) {
-            const uint32_t ta = t_lane + 256 + 64 * j + 16 * grp;
+            const uint32_t ta = t_lane + kTmemO + 64 * j + 16 * grp;
             float v[16];
             tmem_ld16(ta, v);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) v[c] *= a[c];
+            for (int k = 0; k < 16; ++k) v[k] *= a[k];
             tmem_st16(ta, v);
           }
         }
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&bars[kBarOReady + (i & 1)]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarOReady + (i & 1)]);
     }
     // This loop may have run a tile ahead of PV, so the barrier can still be
     // one phase short of tile T-2: wait for that phase first, or the parity
@@ -810,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp >= 4) {
     // ============================================================ epilogue (warps 4-23)
-    // O^T / l -> part_o, the sixteen [128 dims x 16 columns] TMEM chunks
+    // O^T / l -> part_o, the sixteen [128 dims x 16 rows] TMEM chunks
     // spread over the five warpgroups (thread = latent dim of a block)
     tc_fence_after();
     if (*abort_flag == 0) {
@@ -822,20 +853,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row_stride = (int64_t)args.max_splits * 512;
       float* staged = reinterpret_cast<float*>(smem + kOffRing);  // [64][512], ring is free
 #pragma unroll 1
-      for (int c = ewg; c < 16; c += 5) {
-        const int j = c >> 2, grp = c & 3;
+      for (int ch = ewg; ch < 16; ch += 5) {
+        const int j = ch >> 2, grp = ch & 3;
         float v[16];
-        tmem_ld16(t_lane + 256 + 64 * j + 16 * grp, v);
+        tmem_ld16(t_lane + kTmemO + 64 * j + 16 * grp, v);
         if (npieces == 1) {
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const int n = grp * 16 + cc;
-            if (n < rows_valid) po[n * row_stride + 128 * j + d_lane] = v[cc] * sc.inv_l[n];
+          for (int k = 0; k < 16; ++k) {
+            const int nn = grp * 16 + k;
+            if (nn < rows_valid) po[nn * row_stride + 128 * j + d_lane] = v[k] * sc.inv_l[nn];
           }
         } else {
           // unnormalised O, merged across the cluster below
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) staged[(grp * 16 + cc) * 512 + 128 * j + d_lane] = v[cc];
+          for (int k = 0; k < 16; ++k) staged[(grp * 16 + k) * 512 + 128 * j + d_lane] = v[k];
         }
       }
     }
@@ -854,14 +885,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace fp8k
 
 cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fp8k::decode_fp8_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         fp8k::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // the shared-memory opt-in is a per-device attribute of the kernel: set it
+  // on every launch (a cheap host call) so that any device the caller makes
+  // current is configured
+  cudaError_t e = cudaFuncSetAttribute(fp8k::decode_fp8_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       fp8k::kSmemBytes);
+  if (e != cudaSuccess) return e;
   const long long units = (long long)a.groups * a.max_splits * a.B;
   const long long ctas = a.split_from + a.pad + (units - a.split_from) * a.pieces;
   if (a.pieces == 1) {
