@@ -404,21 +404,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) prefetch_tensormap(&kv_map);
     __syncwarp();
     const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
+    // Page ids of this run, 32 at a time (one load per lane instead of a
+    // dependent load per tile): lane l of window w holds block-table entry
+    // pg0 + 32 w + l (-1 past the row).  Two windows are held: the loads of
+    // tile i and the L2 prefetch of tile i + kAhead never span more.
+    auto load_window = [&](int w) -> int {
+      const int k = pg0 + 32 * w + lane;
+      return k < args.max_pages ? bt[k] : -1;
+    };
+    int win = 0;
+    int win_lo = load_window(0), win_hi = load_window(1);
+    auto page_at = [&](int k) -> int {  // run page index k, warp-uniform
+      return __shfl_sync(0xffffffffu, (k >> 5) == win ? win_lo : win_hi, k & 31);
+    };
     // L2 prefetch of a whole tile: each page is one contiguous 36 KiB block,
     // so one untiled bulk prefetch per page; page ids out of range are
     // skipped here and reported by the load path
     auto prefetch_tile = [&](int i) {
       const int tok0 = t0 + i * kTile;
-      const int pa = bt[pg0 + 2 * i];
+      const int pa = page_at(2 * i);
       const bool want_b = tok0 + 64 < t1;
-      const int pb = want_b ? bt[pg0 + 2 * i + 1] : -1;
+      const int pb = page_at(2 * i + 1);
       if (pa >= 0 && (int64_t)pa < args.num_pages)
         bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pa * kPageBytes, kPageBytes);
       if (want_b && pb >= 0 && (int64_t)pb < args.num_pages)
         bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pb * kPageBytes, kPageBytes);
     };
     constexpr int kAhead = 2;  // tiles prefetched into L2 ahead of the one being loaded
-    for (int i = 1; i < min(T, kAhead); ++i) prefetch_tile(i);
     int last_parity[kRingPairs];
     bool armed[kRingPairs];
     for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
@@ -426,11 +438,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int u = 0;  // load number of the next latent pair
     for (int i = 0; i < T && ok; ++i) {
-      if (i + kAhead < T) prefetch_tile(i + kAhead);
+      if ((2 * i) >> 5 > win) {  // the loads moved into the next window
+        win_lo = win_hi;
+        ++win;
+        win_hi = load_window(win + 1);
+      }
+      // tile 0 goes first; tiles 1 .. kAhead are loaded straight away too, so
+      // the L2 prefetch starts with tile kAhead + 1
+      if (i >= 1 && i + kAhead < T) prefetch_tile(i + kAhead);
       const int tok0 = t0 + i * kTile;
-      const int pa = bt[pg0 + 2 * i];
+      const int pa = page_at(2 * i);
       const bool want_b = tok0 + 64 < t1;
-      const int pb = want_b ? bt[pg0 + 2 * i + 1] : 0;
+      const int pb = want_b ? page_at(2 * i + 1) : 0;
       const bool la = pa >= 0 && (int64_t)pa < args.num_pages;
       const bool lb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
       if (lane == 0 && (!la || (want_b && !lb))) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
@@ -594,29 +613,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bar_id = 1 + qd;         // the four warps of this quadrant
     float c_head;                      // softmax_scale * kv_scale * log2(e) * 2^-e
     {
-      // ---- Q -> Q' = [Q_hi ; Q_lo] with a power-of-two scale per query row:
-      // this thread converts latent dims [128c, 128c+128) and RoPE dims
-      // [16c, 16c+16) of row n, term `part`; the latent bytes go to TMEM lane
-      // 32 qd + lane, the RoPE bytes to shared memory row 32 qd + lane.  The
-      // row's amax is taken over all 576 dims (the four slices of the row).
-      const uint16_t* qn = args.q_nope + (row_base + n) * 512 + 128 * c;
-      const uint16_t* qr = args.q_rope + (row_base + n) * 64 + 16 * c;
-      auto load8 = [&](int k) -> uint4 {  // dims 8k .. 8k+7 of the slice (k >= 16: RoPE)
-        if (!valid) return make_uint4(0, 0, 0, 0);
-        return k < 16 ? *reinterpret_cast<const uint4*>(qn + 8 * k)
-                      : *reinterpret_cast<const uint4*>(qr + 8 * (k - 16));
-      };
+      // ---- Q -> Q' = [Q_hi ; Q_lo] with a power-of-two scale per query row.
+      // Row n's slice c is latent dims [128c, 128c+128) and RoPE dims
+      // [16c, 16c+16); the two lanes of the row (l and l ^ 16) each load one
+      // half of it in a single round of loads, compute both terms of their
+      // half, and swap the term the other lane needs.  The latent bytes go to
+      // TMEM lane 32 qd + lane, the RoPE bytes to shared memory row 32 qd +
+      // lane.  The row's amax is taken over all 576 dims (both halves of the
+      // four slices).
+      const uint16_t* qn = args.q_nope + (row_base + n) * 512 + 128 * c + 64 * part;
+      const uint16_t* qr = args.q_rope + (row_base + n) * 64 + 16 * c + 8 * part;
+      uint4 v[9];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        v[k] = valid ? *reinterpret_cast<const uint4*>(qn + 8 * k) : make_uint4(0, 0, 0, 0);
+      v[8] = valid ? *reinterpret_cast<const uint4*>(qr) : make_uint4(0, 0, 0, 0);
       uint32_t amax_bits = 0;
-#pragma unroll 6
-      for (int k = 0; k < 18; ++k) {
-        const uint4 v = load8(k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 9; ++k) {
+        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           amax_bits = max(amax_bits, (w[e] << 16) & 0x7FFFFFFFu);
           amax_bits = max(amax_bits, w[e] & 0x7FFF0000u);
         }
       }
+      amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, 16));
       if (part == 0) sc.red[c][n] = __uint_as_float(amax_bits);
       named_bar_sync(bar_id, 128);
       const float amax = fmaxf(fmaxf(sc.red[0][n], sc.red[1][n]), fmaxf(sc.red[2][n], sc.red[3][n]));
@@ -628,32 +650,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       c_head = valid ? args.qk_scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23) : 0.0f;
       const float sc_up = __uint_as_float((uint32_t)(127 + e) << 23);
-      auto term_of = [&](int k) -> uint2 {  // this thread's term of dims 8k .. 8k+7
-        const uint4 v = load8(k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      // this lane's term of its own 8 dims (mine) and of the partner's 8 dims
+      // of the same position (got), for load k
+      auto terms = [&](int k, uint2& mine, uint2& got) {
+        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
         float x[8];
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
           x[2 * e2] = __uint_as_float(w[e2] << 16) * sc_up;
           x[2 * e2 + 1] = __uint_as_float(w[e2] & 0xFFFF0000u) * sc_up;
         }
-        return term8(x, part != 0);
+        const uint2 hi = term8(x, false), lo = term8(x, true);
+        mine = part ? lo : hi;
+        const uint2 give = part ? hi : lo;  // the partner's term of my dims
+        got.x = __shfl_xor_sync(0xffffffffu, give.x, 16);
+        got.y = __shfl_xor_sync(0xffffffffu, give.y, 16);
       };
       const uint32_t t_q = tmem + ((uint32_t)(32 * qd) << 16) + kTmemQ + 32 * c;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {  // 64 latent dims = 16 TMEM columns at a time
-        float cols[16];
+      {
+        float first[16], second[16];  // slice dims [0, 64) and [64, 128) of this lane's term
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint2 t8 = term_of(8 * h + k);
-          cols[2 * k] = __uint_as_float(t8.x);
-          cols[2 * k + 1] = __uint_as_float(t8.y);
+          uint2 mine, got;
+          terms(k, mine, got);
+          first[2 * k] = __uint_as_float(part ? got.x : mine.x);
+          first[2 * k + 1] = __uint_as_float(part ? got.y : mine.y);
+          second[2 * k] = __uint_as_float(part ? mine.x : got.x);
+          second[2 * k + 1] = __uint_as_float(part ? mine.y : got.y);
         }
-        tmem_st16(t_q + 16 * h, cols);
+        tmem_st16(t_q, first);
+        tmem_st16(t_q + 16, second);
       }
-#pragma unroll
-      for (int k = 16; k < 18; ++k)
-        *reinterpret_cast<uint2*>(smem + kOffQr + sw64(32 * qd + lane, 16 * c + 8 * (k - 16))) = term_of(k);
+      {
+        uint2 mine, got;
+        terms(8, mine, got);
+        const uint2 lo8 = part ? got : mine, hi8 = part ? mine : got;  // RoPE dims 0-7, 8-15 of the slice
+        *reinterpret_cast<uint4*>(smem + kOffQr + sw64(32 * qd + lane, 16 * c)) =
+            make_uint4(lo8.x, lo8.y, hi8.x, hi8.y);
+      }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
