@@ -53,9 +53,10 @@
 // sums are rescaled (by 2^(m_old - m_new)) only for rows whose max moved.
 //
 // Warp roles (768 threads):
-//   warp 0        TMA producer: pages -> 64-byte-swizzled 128-dim pairs in an
-//                 11-slot ring (2.75 tiles) plus a 2-slot RoPE ring, and L2
-//                 prefetch of tiles ahead
+//   warp 0        TMA producer: pages -> 128-byte-swizzled 128-dim pairs
+//                 (one 8 KiB box per page and pair) in an 11-slot ring (2.75
+//                 tiles) plus a 2-slot RoPE ring (64-byte swizzle), each
+//                 tile's pages bulk-prefetched into L2 just before its loads
 //   warp 1        UMMA issuer (warp-uniform polling of readiness, PV before
 //                 QK; one elected lane issues) and TMEM owner
 //   warps 4-19    softmax: warp w works on TMEM lane quadrant w % 4 (16 query
@@ -82,7 +83,6 @@ constexpr int kRows = 64;           // query rows per CTA (UMMA N for PV)
 constexpr int kTile = 128;          // tokens per tile (UMMA N for QK, K for PV)
 constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
-constexpr uint32_t kPageBytes = 64 * 576;  // one page of the pool
 constexpr int kRingPairs = 11;      // latent pair slots: 2.75 tiles in flight
 constexpr int kRopeSlots = 2;
 constexpr float kPShift = 7.0f;     // log2 of the factor carried by the softmax weights
@@ -277,7 +277,8 @@ __device__ __forceinline__ void merge_pieces(int npieces, const DecodeArgs& args
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_fp8_kernel(const DecodeArgs args, const __grid_constant__ CUtensorMap kv_map) {
+    decode_fp8_kernel(const DecodeArgs args, const __grid_constant__ CUtensorMap kv_map,
+                      const __grid_constant__ CUtensorMap rope_map) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Scratch& sc = *reinterpret_cast<Scratch*>(smem + kOffScratch);
   const int tid = threadIdx.x;
@@ -304,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = unit % args.groups;
   const int s = (unit / args.groups) % args.max_splits;
   const int b = unit / (args.groups * args.max_splits);
-
   // ---------------------------------------------------------------- split range (step A2)
   const int L = args.seq_lens[b];
   const int S_b = args.num_splits[b];
@@ -401,13 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // lane issues each TMA instruction and barrier arrival.  Latent pair j of
     // tile i is load number u = 4 i + j and goes to ring slot u % 11; the
     // RoPE chunk of tile i goes to slot i % 2 of its own ring.
-    if (lane == 0) prefetch_tensormap(&kv_map);
+    if (lane == 0) {
+      prefetch_tensormap(&kv_map);
+      prefetch_tensormap(&rope_map);
+    }
     __syncwarp();
     const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
     // Page ids of this run, 32 at a time (one load per lane instead of a
     // dependent load per tile): lane l of window w holds block-table entry
-    // pg0 + 32 w + l (-1 past the row).  Two windows are held: the loads of
-    // tile i and the L2 prefetch of tile i + kAhead never span more.
+    // pg0 + 32 w + l (-1 past the row); the next window is loaded ahead.
     auto load_window = [&](int w) -> int {
       const int k = pg0 + 32 * w + lane;
       return k < args.max_pages ? bt[k] : -1;
@@ -417,9 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto page_at = [&](int k) -> int {  // run page index k, warp-uniform
       return __shfl_sync(0xffffffffu, (k >> 5) == win ? win_lo : win_hi, k & 31);
     };
-    // L2 prefetch of a whole tile: each page is one contiguous 36 KiB block,
-    // so one untiled bulk prefetch per page; page ids out of range are
-    // skipped here and reported by the load path
+    // An untiled bulk L2 prefetch of each of the tile's two pages (36 KiB
+    // contiguous each) right before the tile's TMA loads: measured a little
+    // faster than the TMA loads alone, and faster than prefetching further
+    // ahead (which only adds to the queues in front of the loads).
+    constexpr uint32_t kPageBytes = 64 * 576;
     auto prefetch_tile = [&](int i) {
       const int tok0 = t0 + i * kTile;
       const int pa = page_at(2 * i);
@@ -430,7 +434,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (want_b && pb >= 0 && (int64_t)pb < args.num_pages)
         bulk_prefetch_l2_elect(args.kv_pages + (int64_t)pb * kPageBytes, kPageBytes);
     };
-    constexpr int kAhead = 2;  // tiles prefetched into L2 ahead of the one being loaded
     int last_parity[kRingPairs];
     bool armed[kRingPairs];
     for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
@@ -443,9 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++win;
         win_hi = load_window(win + 1);
       }
-      // tile 0 goes first; tiles 1 .. kAhead are loaded straight away too, so
-      // the L2 prefetch starts with tile kAhead + 1
-      if (i >= 1 && i + kAhead < T) prefetch_tile(i + kAhead);
+      prefetch_tile(i);
       const int tok0 = t0 + i * kTile;
       const int pa = page_at(2 * i);
       const bool want_b = tok0 + 64 < t1;
@@ -453,7 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool la = pa >= 0 && (int64_t)pa < args.num_pages;
       const bool lb = want_b && pb >= 0 && (int64_t)pb < args.num_pages;
       if (lane == 0 && (!la || (want_b && !lb))) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
-      const uint32_t bytes_chunk = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
+      const uint32_t bytes_pair = (la ? 8192u : 0u) + (lb ? 8192u : 0u);  // 128 dims of both pages
+      const uint32_t bytes_rope = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
       for (int j = 0; j < 4; ++j, ++u) {
         const int slot = u % kRingPairs;
         const int use = u / kRingPairs;  // how many times the slot was filled before
@@ -464,16 +466,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t* full = &bars[kBarFull + slot];
         if (args.inject_stall && i == 0 && j == 0 && blockIdx.x == 0)
           continue;  // test hook: this slot is never armed, so its waits run out
-        mbar_arrive_expect_tx_elect(full, 2 * bytes_chunk);
+        mbar_arrive_expect_tx_elect(full, bytes_pair);
         armed[slot] = true;
         last_parity[slot] = use & 1;
+        // latent dims [128 j, 128 j + 128) of the tile: [128 tokens][128 B],
+        // 128-byte swizzle, the second page's 64 tokens 8 KiB in
         uint8_t* dst = smem + kOffRing + slot * kPair;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int chunk = 2 * j + cc;
-          if (la) tma_load_3d_elect(dst + cc * kChunk, &kv_map, full, chunk * 64, 0, pa);
-          if (lb) tma_load_3d_elect(dst + cc * kChunk + 4096, &kv_map, full, chunk * 64, 0, pb);
-        }
+        if (la) tma_load_3d_elect(dst, &kv_map, full, 128 * j, 0, pa);
+        if (lb) tma_load_3d_elect(dst + 8192, &kv_map, full, 128 * j, 0, pb);
       }
       if (!ok) break;
       const int rs = i % kRopeSlots;
@@ -483,11 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       uint64_t* rfull = &bars[kBarRopeFull + rs];
-      mbar_arrive_expect_tx_elect(rfull, bytes_chunk);
+      mbar_arrive_expect_tx_elect(rfull, bytes_rope);
       rope_last[rs] = i;
       uint8_t* rdst = smem + kOffRope + rs * kChunk;
-      if (la) tma_load_3d_elect(rdst, &kv_map, rfull, 512, 0, pa);
-      if (lb) tma_load_3d_elect(rdst + 4096, &kv_map, rfull, 512, 0, pb);
+      if (la) tma_load_3d_elect(rdst, &rope_map, rfull, 512, 0, pa);
+      if (lb) tma_load_3d_elect(rdst + 4096, &rope_map, rfull, 512, 0, pb);
     }
     // drain: every armed transaction has landed before the CTA may exit
     const uint64_t t_start = globaltimer_ns();
@@ -506,13 +506,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warp-uniform scheduler; one elected lane issues each MMA and commit.
     const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, 128, 128);  // E4M3, A K-major (TMEM or smem), B K-major, N=128
     const uint32_t idesc_pv = instr_desc(0, 0, 1, 0, 128, 64);   // A MN-major, B K-major, N=64
-    // K-major SW64 (8-row groups 512 B apart), MN-major SW64 (64-element
-    // atoms 8 KiB apart, 8-row groups 512 B apart), K-major SW128 (8-row
-    // groups 1 KiB apart) descriptor bases
-    const uint64_t dRingK = smem_desc(smem_u32(smem + kOffRing), 16, 512, 4);
+    // Latent pairs are [128 tokens][128 B] with the 128-byte swizzle: K-major
+    // for QK (8-row groups 1 KiB apart) and MN-major for PV (one 128-dim atom
+    // across M, 8-token groups 1 KiB apart).  The RoPE chunks and the Q' RoPE
+    // operand are K-major with the 64-byte swizzle (8-row groups 512 B apart);
+    // P is K-major with the 128-byte swizzle.
+    const uint64_t dRingK = smem_desc(smem_u32(smem + kOffRing), 16, 1024, 2);
     const uint64_t dRope = smem_desc(smem_u32(smem + kOffRope), 16, 512, 4);
     const uint64_t dQr = smem_desc(smem_u32(smem + kOffQr), 16, 512, 4);
-    const uint64_t dRingMN = smem_desc(smem_u32(smem + kOffRing), kChunk, 512, 4);
+    const uint64_t dRingMN = smem_desc(smem_u32(smem + kOffRing), kPair, 1024, 2);
     const uint64_t dPhi = smem_desc(smem_u32(smem + kOffPhi), 16, 1024, 2);
     const uint64_t dPlo = smem_desc(smem_u32(smem + kOffPlo), 16, 1024, 2);
     const uint32_t d_s = tmem + kTmemS;
@@ -537,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = (4 * np + j) % kRingPairs;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = desc_at(dRingMN, slot * kPair + kk * 2048);
+            const uint64_t a = desc_at(dRingMN, slot * kPair + kk * 4096);  // tokens 32 kk ..
             umma_f8_fill_elect(tmem + kTmemO + 64 * j, a, desc_at(dPhi, kk * 32), idesc_pv,
                                (np > 0 || kk > 0) ? 1u : 0u);
             umma_f8_lastuse_elect(tmem + kTmemO + 64 * j, a, desc_at(dPlo, kk * 32), idesc_pv, 1u);
@@ -561,13 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t b_off = ((4 * nq + qpair) % kRingPairs) * kPair;
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const int ks = 4 * qpair + 2 * cc + kk;  // K step of 32 latent dims
-              umma_f8_ts_elect(d_s, tmem + kTmemQ + 8 * ks, desc_at(dRingK, b_off + cc * kChunk + kk * 32),
-                               idesc_qk, ks != 0 ? 1u : 0u);
-            }
+          for (int kk = 0; kk < 4; ++kk) {
+            const int ks = 4 * qpair + kk;  // K step of 32 latent dims
+            umma_f8_ts_elect(d_s, tmem + kTmemQ + 8 * ks, desc_at(dRingK, b_off + kk * 32), idesc_qk,
+                             ks != 0 ? 1u : 0u);
+          }
           ++qpair;
           progress = true;
         }
@@ -785,12 +785,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = tid_s & 127;
         if (t0 + i * kTile + r >= t1) {
           const int slot = (4 * i + (tid_s >> 7)) % kRingPairs;
+          uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + slot * kPair + r * 128);
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint4* row = reinterpret_cast<uint4*>(smem + kOffRing + slot * kPair + cc * kChunk + r * 64);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) row[k] = make_uint4(0, 0, 0, 0);
-          }
+          for (int k = 0; k < 8; ++k) row[k] = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
@@ -918,7 +915,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace fp8k
 
-cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cudaStream_t stream) {
+cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map,
+                              const CUtensorMap& rope_map, cudaStream_t stream) {
   // the shared-memory opt-in is a per-device attribute of the kernel: set it
   // on every launch (a cheap host call) so that any device the caller makes
   // current is configured
@@ -929,7 +927,8 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cu
   const long long units = (long long)a.groups * a.max_splits * a.B;
   const long long ctas = a.split_from + a.pad + (units - a.split_from) * a.pieces;
   if (a.pieces == 1) {
-    fp8k::decode_fp8_kernel<<<(unsigned)ctas, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map);
+    fp8k::decode_fp8_kernel<<<(unsigned)ctas, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map,
+                                                                                         rope_map);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -947,7 +946,7 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cu
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fp8k::decode_fp8_kernel, a, kv_map);
+  return cudaLaunchKernelEx(&cfg, fp8k::decode_fp8_kernel, a, kv_map, rope_map);
 }
 
 }  // namespace mla

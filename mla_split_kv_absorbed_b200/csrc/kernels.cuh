@@ -51,9 +51,12 @@ struct DecodeArgs {
   int inject_stall;     // test hook: leave the first load of CTA (0, 0, 0) unissued
 };
 
-// FP8 E4M3 cache: kv_map is a 3-D tiled TMA map over kv_pages viewed as
-// [num_pages][64][576] bytes, box {64 B, 64 rows, 1 page}, 64-byte swizzle.
-cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map, cudaStream_t stream);
+// FP8 E4M3 cache: kv_map and rope_map are 3-D tiled TMA maps over kv_pages
+// viewed as [num_pages][64][576] bytes: kv_map with box {128 B, 64 rows,
+// 1 page} and the 128-byte swizzle (the latent dims), rope_map with box
+// {64 B, 64 rows, 1 page} and the 64-byte swizzle (the RoPE dims).
+cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map,
+                              const CUtensorMap& rope_map, cudaStream_t stream);
 
 // bf16 cache: kv_map over [num_pages][64][576] bf16, box {64 elems, 64 rows,
 // 1 page}, 128-byte swizzle.

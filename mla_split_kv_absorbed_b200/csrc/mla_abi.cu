@@ -62,23 +62,21 @@ EncodeTiledFn encode_fn() {
 }
 
 // TMA map over kv_pages viewed as [num_pages][64][576] elements with a box of
-// {64 elements, 64 rows, 1 page}: 64 B rows (64-byte swizzle) for E4M3,
-// 128 B rows (128-byte swizzle) for bf16.
-int make_kv_map(CUtensorMap* map, const void* kv_pages, int kv_dtype, int64_t num_pages) {
+// {box_x elements, 64 rows, 1 page} and the given swizzle.
+int make_kv_map(CUtensorMap* map, const void* kv_pages, int kv_dtype, int64_t num_pages,
+                cuuint32_t box_x, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return MLA_ERR_CUDA;
   const cuuint64_t esz = kv_dtype == MLA_KV_FP8_E4M3 ? 1 : 2;
   const cuuint64_t dims[3] = {(cuuint64_t)kRow, (cuuint64_t)kPage, (cuuint64_t)num_pages};
   const cuuint64_t strides[2] = {kRow * esz, (cuuint64_t)kPage * kRow * esz};
-  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t box[3] = {box_x, 64, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map,
                         kv_dtype == MLA_KV_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                     : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                         3, const_cast<void*>(kv_pages), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        kv_dtype == MLA_KV_FP8_E4M3 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                    : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_INVALID_ARG;
 }
@@ -157,10 +155,19 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
   if (q_len > 4 || q_len * H > 512 || max_splits > 256 || B > 65535 || (q_len * H) % 16 != 0)
     return MLA_ERR_UNSUPPORTED;
 
-  CUtensorMap map;
+  // FP8: the latent dims as 128-byte rows (128-byte swizzle) and the RoPE dims
+  // as 64-byte rows (64-byte swizzle); bf16: 64-element (128-byte) rows
+  CUtensorMap map, rope_map;
   std::memset(&map, 0, sizeof(map));
-  int st = make_kv_map(&map, kv_pages, kv_dtype, num_pages);
+  std::memset(&rope_map, 0, sizeof(rope_map));
+  int st = kv_dtype == MLA_KV_FP8_E4M3
+               ? make_kv_map(&map, kv_pages, kv_dtype, num_pages, 128, CU_TENSOR_MAP_SWIZZLE_128B)
+               : make_kv_map(&map, kv_pages, kv_dtype, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != MLA_OK) return st;
+  if (kv_dtype == MLA_KV_FP8_E4M3) {
+    st = make_kv_map(&rope_map, kv_pages, kv_dtype, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != MLA_OK) return st;
+  }
 
   mla::DecodeArgs a = {};
   a.q_nope = q_nope;
@@ -190,7 +197,7 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
     a.pad = plan[3];
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, s)
+  return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, rope_map, s)
                                                : mla::launch_decode_bf16(a, map, s));
 }
 
