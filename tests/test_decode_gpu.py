@@ -5,7 +5,8 @@ q_len 1-4 with causal masking (one query position per row group, and four
 positions inside one group), 16 to 128 heads and NaN-poisoned pages around
 the visible range.  Small grids exercise the cluster path in which every
 split is cut across 2 or 4 CTAs; one case has a partly filled last wave whose
-units alone are cut.  The full-size cases run the benchmark workloads in the
+units alone are cut, and larger grids run several waves with or without such a
+cut tail.  The full-size cases run the benchmark workloads in the
 benchmark's launch configuration and compare sampled rows.
 """
 import numpy as np
@@ -34,6 +35,15 @@ SMALL = [
     # 5 x 32 = 160 (group, split) units on 148 SMs: the last, partly filled
     # wave (12 units) is cut into 2-CTA clusters; short splits give empty pieces
     ("b16_128k_fp8", dict(seq_lens=[5000, 3000, 64, 4100, 777], splits=32)),
+    # 310 units on 148 SMs: two full waves, then 14 one-tile units cut in 2
+    # whose second pieces are empty
+    ("b16_128k_fp8", dict(seq_lens=[3000, 2500, 700, 4100, 64, 1800, 2222, 3333, 900, 3900],
+                          splits=31)),
+    # q_len 4, 4 row groups: 208 units = one full wave + 60 units cut in 2
+    ("verify_q4_256k_fp8", dict(seq_lens=[3000, 2000, 900, 4100], splits=13, H=64)),
+    # 396 units: two full waves + 100, no cut
+    ("b16_128k_fp8", dict(seq_lens=[2100, 3000, 130, 4000, 2500, 1, 3900, 2048, 640, 3500, 1200,
+                                    2900], splits=33)),
 ]
 
 
