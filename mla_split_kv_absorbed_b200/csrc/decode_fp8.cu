@@ -20,11 +20,11 @@
 // operands E4M3.  Q (bf16, 8 significant bits) is scaled per row by a power
 // of two and split as Q = Q_hi + Q_lo with Q_hi = Q rounded to 4 significant
 // bits and Q_lo = E4M3(Q - Q_hi); this is exact for every element within a
-// factor 2^-9 of the row maximum.  The softmax weights are scaled by 2^7,
-// p' = 2^(s - m + 7), and split the same way, P = P_hi + P_lo: about 8
-// significant bits (like bf16) for every p' >= 2^-2 and an absolute error of
-// at most 2^-9 for smaller weights.  The scale cancels in O / l and is removed
-// from the LSE.
+// factor 2^-9 of the row maximum.  The softmax weights are scaled by 2^4,
+// p' = 2^(s - m + 4), and split the same way, P = P_hi + P_lo: about 8
+// significant bits (like bf16) for every p' >= 2^-1 and an absolute error of
+// at most 2^-10 for smaller weights, while the largest weight of a row is at
+// least 2^4.  The scale cancels in O / l and is removed from the LSE.
 //
 // Tensor-core mapping.  QK^T takes the 128 two-term query rows as M and the
 // 128 tokens of a tile as N:
@@ -46,7 +46,7 @@
 //
 // Online softmax (log2 domain, scores pre-multiplied by log2 e), with a lazy
 // running max: the max m used for a row only moves when a tile's max exceeds
-// it by more than 1.75 (log2 units), so p' stays <= 2^8.75 < 448, the E4M3
+// it by more than 4.75 (log2 units), so p' stays <= 2^8.75 < 448, the E4M3
 // maximum.  A tile in which no score of a quadrant's rows exceeds its max by
 // that much (the common case once the max has settled) skips the max
 // reduction altogether: one barrier vote decides it.  O^T columns and row
@@ -56,9 +56,12 @@
 //   warp 0        TMA producer: pages -> 128-byte-swizzled 128-dim pairs
 //                 (one 8 KiB box per page and pair) in an 11-slot ring (2.75
 //                 tiles) plus a 2-slot RoPE ring (64-byte swizzle), each
-//                 tile's pages bulk-prefetched into L2 just before its loads
-//   warp 1        UMMA issuer (warp-uniform polling of readiness, PV before
-//                 QK; one elected lane issues) and TMEM owner
+//                 tile's pages bulk-prefetched into L2 just before its loads,
+//                 its RoPE chunk loaded before its latent pairs
+//   warp 1        UMMA issuer (warp-uniform polling of readiness; the QK
+//                 MMAs whose operands have landed go before a ready PV, which
+//                 measured faster than the reverse; one elected lane issues)
+//                 and TMEM owner
 //   warps 4-19    softmax: warp w works on TMEM lane quadrant w % 4 (16 query
 //                 rows) and token slice (w - 4) / 4 (32 tokens of the tile)
 //   warps 20-23   O^T rescaling between tiles (thread = latent dim)
@@ -85,8 +88,8 @@ constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
 constexpr int kRingPairs = 11;      // latent pair slots: 2.75 tiles in flight
 constexpr int kRopeSlots = 2;
-constexpr float kPShift = 7.0f;     // log2 of the factor carried by the softmax weights
-constexpr float kLazy = 1.75f;      // the used max moves only when exceeded by more than this
+constexpr float kPShift = 4.0f;     // log2 of the factor carried by the softmax weights
+constexpr float kLazy = 4.75f;      // the used max moves only when exceeded by more than this
 
 constexpr int kOffRing = 0;                                  // 11 pairs
 constexpr int kOffRope = kOffRing + kRingPairs * kPair;      // 180224: 2 RoPE chunks
@@ -456,6 +459,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && (!la || (want_b && !lb))) set_error(args.dev_error, MLA_DEVERR_BAD_PAGE);
       const uint32_t bytes_pair = (la ? 8192u : 0u) + (lb ? 8192u : 0u);  // 128 dims of both pages
       const uint32_t bytes_rope = (la ? 4096u : 0u) + (lb ? 4096u : 0u);
+      const int rs = i % kRopeSlots;
+      if (i >= kRopeSlots) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars[kBarRopeEmpty + rs], ((i / kRopeSlots) - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      uint64_t* rfull = &bars[kBarRopeFull + rs];
+      mbar_arrive_expect_tx_elect(rfull, bytes_rope);
+      rope_last[rs] = i;
+      uint8_t* rdst = smem + kOffRope + rs * kChunk;
+      if (la) tma_load_3d_elect(rdst, &rope_map, rfull, 512, 0, pa);
+      if (lb) tma_load_3d_elect(rdst + 4096, &rope_map, rfull, 512, 0, pb);
       for (int j = 0; j < 4; ++j, ++u) {
         const int slot = u % kRingPairs;
         const int use = u / kRingPairs;  // how many times the slot was filled before
@@ -476,18 +491,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lb) tma_load_3d_elect(dst + 8192, &kv_map, full, 128 * j, 0, pb);
       }
       if (!ok) break;
-      const int rs = i % kRopeSlots;
-      if (i >= kRopeSlots) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars[kBarRopeEmpty + rs], ((i / kRopeSlots) - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-      uint64_t* rfull = &bars[kBarRopeFull + rs];
-      mbar_arrive_expect_tx_elect(rfull, bytes_rope);
-      rope_last[rs] = i;
-      uint8_t* rdst = smem + kOffRope + rs * kChunk;
-      if (la) tma_load_3d_elect(rdst, &rope_map, rfull, 512, 0, pa);
-      if (lb) tma_load_3d_elect(rdst + 4096, &rope_map, rfull, 512, 0, pb);
     }
     // drain: every armed transaction has landed before the CTA may exit
     const uint64_t t_start = globaltimer_ns();
@@ -524,12 +527,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarQReady], 0, abort_flag));
     tc_fence_after();
     int nq = 0, qpair = 0, np = 0;
-    bool s_free = false;
+    bool s_free = false, rope_done = false;
     uint64_t idle_since = 0;
     uint32_t idle_spins = 0;
     while (ok && np < T) {
       bool progress = false;
-      // ---------------- O^T += V(np)^T . (P_hi + P_lo), before any further QK
+      // ---------------- S'(nq) = Q' . K(nq)^T, one 128-dim pair at a time
+      if (nq < T) {
+        if (!s_free) {
+          s_free = nq < 1 || ready(kBarSEmpty, (nq - 1) & 1);
+          if (s_free) tc_fence_after();
+        }
+        // the RoPE chunk (loaded first) goes first when it has landed; the
+        // first MMA of a tile starts S' afresh
+        if (s_free && !rope_done && ready(kBarRopeFull + nq % kRopeSlots, (nq / kRopeSlots) & 1)) {
+          tc_fence_after();
+          const uint32_t r_off = (nq % kRopeSlots) * kChunk;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            umma_f8_elect(d_s, desc_at(dQr, kk * 32), desc_at(dRope, r_off + kk * 32), idesc_qk,
+                          (qpair > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_elect(&bars[kBarRopeEmpty + nq % kRopeSlots]);
+          rope_done = true;
+          progress = true;
+        }
+        while (s_free && qpair < 4 &&
+               ready(kBarFull + (4 * nq + qpair) % kRingPairs, ((4 * nq + qpair) / kRingPairs) & 1)) {
+          tc_fence_after();
+          const uint32_t b_off = ((4 * nq + qpair) % kRingPairs) * kPair;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int ks = 4 * qpair + kk;  // K step of 32 latent dims
+            umma_f8_ts_elect(d_s, tmem + kTmemQ + 8 * ks, desc_at(dRingK, b_off + kk * 32), idesc_qk,
+                             (rope_done || ks != 0) ? 1u : 0u);
+          }
+          ++qpair;
+          progress = true;
+        }
+        if (s_free && qpair == 4 && rope_done) {
+          umma_commit_elect(&bars[kBarSFull]);
+          ++nq;
+          qpair = 0;
+          rope_done = false;
+          s_free = false;
+          progress = true;
+        }
+      }
+      // ---------------- O^T += V(np)^T . (P_hi + P_lo), after any QK that was ready
       if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady + (np & 1), (np >> 1) & 1)) {
         tc_fence_after();
         // block by block, so each latent pair can be refilled as soon as its
@@ -551,39 +595,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit_elect(&bars[kBarPvDone]);
         ++np;
         progress = true;
-      }
-      // ---------------- S'(nq) = Q' . K(nq)^T, one 128-dim pair at a time
-      if (nq < T) {
-        if (!s_free) {
-          s_free = nq < 1 || ready(kBarSEmpty, (nq - 1) & 1);
-          if (s_free) tc_fence_after();
-        }
-        while (s_free && qpair < 4 &&
-               ready(kBarFull + (4 * nq + qpair) % kRingPairs, ((4 * nq + qpair) / kRingPairs) & 1)) {
-          tc_fence_after();
-          const uint32_t b_off = ((4 * nq + qpair) % kRingPairs) * kPair;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int ks = 4 * qpair + kk;  // K step of 32 latent dims
-            umma_f8_ts_elect(d_s, tmem + kTmemQ + 8 * ks, desc_at(dRingK, b_off + kk * 32), idesc_qk,
-                             ks != 0 ? 1u : 0u);
-          }
-          ++qpair;
-          progress = true;
-        }
-        if (s_free && qpair == 4 && ready(kBarRopeFull + nq % kRopeSlots, (nq / kRopeSlots) & 1)) {
-          tc_fence_after();
-          const uint32_t r_off = (nq % kRopeSlots) * kChunk;
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            umma_f8_elect(d_s, desc_at(dQr, kk * 32), desc_at(dRope, r_off + kk * 32), idesc_qk, 1u);
-          umma_commit_elect(&bars[kBarSFull]);
-          umma_commit_elect(&bars[kBarRopeEmpty + nq % kRopeSlots]);
-          ++nq;
-          qpair = 0;
-          s_free = false;
-          progress = true;
-        }
       }
       if (progress) {
         idle_spins = 0;
@@ -763,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
       }
-      // weights carry a 2^7 factor: p' = 2^(s - m + 7) <= 2^8.75
+      // weights carry a 2^4 factor: p' = 2^(s - m + 4) <= 2^8.75
       float pv[16];
       float psum = 0.0f;
 #pragma unroll
