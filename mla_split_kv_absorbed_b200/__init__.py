@@ -11,6 +11,9 @@ Entry points (same names as the C ABI):
 * ``mla_quantize_fp8(x_bf16, y_u8, inv_scale)`` — step A1, saturating E4M3.
 * ``mla_decode_partial(...)`` — steps A2-A8, per-split partial O and LSE.
 * ``mla_combine(...)`` — step A9, log-sum-exp merge into bf16 O and fp32 LSE.
+* ``mla_decode_fused(...)`` — steps A2-A9 in one cooperative launch (FP8, grids
+  that fit on the GPU at once, e.g. batch 1); ``mla_fused_workspace_bytes`` and
+  ``alloc_fused_workspace`` size and zero its workspace.
 * ``mla_partial_workspace_bytes``, ``mla_choose_splits``, ``mla_status_string``.
 * ``mla_append_kv_fp8(...)`` — the KV-append step before the path: RoPE on the
   64-wide key, saturating E4M3 and the paged write in one kernel;
@@ -46,7 +49,7 @@ EXPORTS = ("mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partia
            "mla_combine", "mla_choose_splits", "mla_device_error_status", "mla_status_string",
            "mla_decode_noalloc", "mla_partial_grid", "mla_debug_inject_stall",
            "mla_append_kv_fp8", "mla_rope_cos_sin_table", "mla_combine_f32",
-           "mla_merge_rank_partials")
+           "mla_merge_rank_partials", "mla_fused_workspace_bytes", "mla_decode_fused")
 
 
 class MlaError(RuntimeError):
@@ -99,6 +102,11 @@ def _load_lib():
     lib.mla_device_error_status.restype = i32
     lib.mla_debug_inject_stall.argtypes = [i32]
     lib.mla_debug_inject_stall.restype = i32
+    lib.mla_fused_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.mla_fused_workspace_bytes.restype = ctypes.c_size_t
+    lib.mla_decode_fused.argtypes = [P, P, P, i32, f32, i64, P, i32, P, P, i32, i32, i32, i32,
+                                     f32, P, P, P, P, P]
+    lib.mla_decode_fused.restype = i32
     return lib
 
 
@@ -182,6 +190,44 @@ def mla_decode_partial(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens
         int(max_splits), B, q_len, H, float(softmax_scale),
         _dev(part_o, "part_o", torch.float32), _dev(part_lse, "part_lse", torch.float32),
         None if dev_error is None else _dev(dev_error, "dev_error", torch.int32), _stream(stream)))
+
+
+def mla_fused_workspace_bytes(B: int, q_len: int, H: int, max_splits: int) -> int:
+    return int(_lib.mla_fused_workspace_bytes(B, q_len, H, max_splits))
+
+
+def alloc_fused_workspace(B, q_len, H, max_splits, device="cuda"):
+    """Workspace of mla_decode_fused, zeroed (its two counters must start at zero)."""
+    return torch.zeros(mla_fused_workspace_bytes(B, q_len, H, max_splits), dtype=torch.uint8,
+                       device=device)
+
+
+def mla_decode_fused(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits,
+                     max_splits, softmax_scale, workspace, out, out_lse=None, dev_error=None,
+                     stream=None):
+    """Single-launch decode (FP8 cache, grids that fit on the GPU at once); raises MlaError
+    with MLA_ERR_UNSUPPORTED for other shapes."""
+    B, q_len, H, dl = q_nope.shape
+    if dl != 512 or tuple(q_rope.shape) != (B, q_len, H, 64):
+        raise ValueError("q_nope must be [B][q_len][H][512] and q_rope [B][q_len][H][64]")
+    if kv_pages.dtype != torch.uint8 or kv_pages.dim() != 3 or tuple(kv_pages.shape[1:]) != (64, 576):
+        raise ValueError("kv_pages must be uint8 (E4M3 codes) [num_pages][64][576]")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B][max_pages]")
+    if workspace.numel() * workspace.element_size() < mla_fused_workspace_bytes(B, q_len, H, max_splits):
+        raise ValueError("workspace is too small")
+    if tuple(out.shape) != (B, q_len, H, 512):
+        raise ValueError("out must be [B][q_len][H][512]")
+    _check("mla_decode_fused", _lib.mla_decode_fused(
+        _dev(q_nope, "q_nope", torch.bfloat16), _dev(q_rope, "q_rope", torch.bfloat16),
+        _dev(kv_pages, "kv_pages"), MLA_KV_FP8_E4M3, float(kv_scale), kv_pages.shape[0],
+        _dev(block_table, "block_table", torch.int32), block_table.shape[1],
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(num_splits, "num_splits", torch.int32),
+        int(max_splits), B, q_len, H, float(softmax_scale), _dev(workspace, "workspace"),
+        _dev(out, "out", torch.bfloat16),
+        None if out_lse is None else _dev(out_lse, "out_lse", torch.float32),
+        None if dev_error is None else _dev(dev_error, "dev_error", torch.int32), _stream(stream)))
+    return out
 
 
 def mla_combine(part_o, part_lse, num_splits, max_splits, out, out_lse=None, stream=None):

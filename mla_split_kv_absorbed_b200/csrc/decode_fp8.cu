@@ -123,7 +123,8 @@ struct Scratch {
   uint64_t bars[40];
   uint32_t tmem_base;
   int abort;
-  int pad[2];
+  int merge_fail;            // single-launch mode: the grid barrier timed out
+  int pad;
   float red[4][64];          // per token slice, per query row: amax, tile max, row sums
   float m_run[64];           // max used per query row (log2 units), for the epilogue/merge
   float inv_l[64];           // per query row: kv_scale / l (0 when l == 0), or raw l when cut
@@ -279,10 +280,10 @@ __device__ __forceinline__ void merge_pieces(int npieces, const DecodeArgs& args
     merge_pieces<4>(args, smem, sc, row_base, rows_valid, s);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    decode_fp8_kernel(const DecodeArgs args, const __grid_constant__ CUtensorMap kv_map,
-                      const __grid_constant__ CUtensorMap rope_map) {
-  extern __shared__ __align__(1024) uint8_t smem[];
+// Steps A2-A8 for one CTA: its piece of one unit.  Every early return is
+// uniform across the CTA.
+__device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUtensorMap* kv_map,
+                                             const CUtensorMap* rope_map, uint8_t* smem) {
   Scratch& sc = *reinterpret_cast<Scratch*>(smem + kOffScratch);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -305,6 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     piece = j % args.pieces;  // this CTA's run of the split's tiles
     npieces = args.pieces;
   }
+  // Where this CTA's partial goes: split s of its rows, or, in the
+  // single-launch mode, entry s * pieces + piece of its rows (every piece
+  // writes its own normalised partial, merged with the rest after the grid
+  // barrier; no cluster merge).
+  const bool own = npieces == 1 || args.fused;
   const int g = unit % args.groups;
   const int s = (unit / args.groups) % args.max_splits;
   const int b = unit / (args.groups * args.max_splits);
@@ -331,15 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t0s = p0 * 64;                         // the split's tokens [t0s, t1s)
   const int t1s = min(p1 * 64, vis_base + q_max);
   const int64_t row_base = (int64_t)b * QH + r0;
+  const int slots = args.fused ? args.max_splits * args.pieces : args.max_splits;  // per row
+  const int slot = args.fused ? s * npieces + piece : s;
+  // an empty partial: O = 0, LSE = -inf
+  auto write_empty = [&]() {
+    for (int i = tid; i < rows_valid * 512; i += kThreads) {
+      const int n = i >> 9;
+      args.part_o[((row_base + n) * slots + slot) * 512 + (i & 511)] = 0.0f;
+    }
+    if (tid < rows_valid) args.part_lse[(row_base + tid) * slots + slot] = -INFINITY;
+  };
 
   if (t1s <= t0s) {  // empty split for every row of the group
-    if (piece == 0) {
-      for (int i = tid; i < rows_valid * 512; i += kThreads) {
-        const int n = i >> 9;
-        args.part_o[((row_base + n) * args.max_splits + s) * 512 + (i & 511)] = 0.0f;
-      }
-      if (tid < rows_valid) args.part_lse[(row_base + tid) * args.max_splits + s] = -INFINITY;
-    }
+    if (piece == 0 || args.fused) write_empty();
     return;
   }
   // this CTA's run: tiles [tile0, tile0 + T) of the split's Ts tiles
@@ -354,6 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- setup
   if ((smem_u32(smem) & 1023u) != 0) {  // same for every CTA of the grid
     if (tid == 0) set_error(args.dev_error, MLA_DEVERR_SMEM_ALIGN);
+    return;
+  }
+  if (T == 0 && args.fused) {  // no tiles in this piece: an empty entry
+    write_empty();
     return;
   }
   if (T == 0) {
@@ -405,8 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile i is load number u = 4 i + j and goes to ring slot u % 11; the
     // RoPE chunk of tile i goes to slot i % 2 of its own ring.
     if (lane == 0) {
-      prefetch_tensormap(&kv_map);
-      prefetch_tensormap(&rope_map);
+      prefetch_tensormap(kv_map);
+      prefetch_tensormap(rope_map);
     }
     __syncwarp();
     const int32_t* bt = args.block_table + (int64_t)b * args.max_pages;
@@ -469,8 +483,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx_elect(rfull, bytes_rope);
       rope_last[rs] = i;
       uint8_t* rdst = smem + kOffRope + rs * kChunk;
-      if (la) tma_load_3d_elect(rdst, &rope_map, rfull, 512, 0, pa);
-      if (lb) tma_load_3d_elect(rdst + 4096, &rope_map, rfull, 512, 0, pb);
+      if (la) tma_load_3d_elect(rdst, rope_map, rfull, 512, 0, pa);
+      if (lb) tma_load_3d_elect(rdst + 4096, rope_map, rfull, 512, 0, pb);
       for (int j = 0; j < 4; ++j, ++u) {
         const int slot = u % kRingPairs;
         const int use = u / kRingPairs;  // how many times the slot was filled before
@@ -487,8 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // latent dims [128 j, 128 j + 128) of the tile: [128 tokens][128 B],
         // 128-byte swizzle, the second page's 64 tokens 8 KiB in
         uint8_t* dst = smem + kOffRing + slot * kPair;
-        if (la) tma_load_3d_elect(dst, &kv_map, full, 128 * j, 0, pa);
-        if (lb) tma_load_3d_elect(dst + 8192, &kv_map, full, 128 * j, 0, pb);
+        if (la) tma_load_3d_elect(dst, kv_map, full, 128 * j, 0, pa);
+        if (lb) tma_load_3d_elect(dst + 8192, kv_map, full, 128 * j, 0, pb);
       }
       if (!ok) break;
     }
@@ -815,10 +829,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = (sc.red[0][n] + sc.red[1][n]) + (sc.red[2][n] + sc.red[3][n]);
         const bool nonempty = !bad && l > 0.0f;
         sc.m_run[n] = m_run;
-        if (npieces == 1) {
+        if (own) {
           sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
           if (valid)
-            args.part_lse[(row_base + n) * args.max_splits + s] =
+            args.part_lse[(row_base + n) * slots + slot] =
                 nonempty ? (m_run - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
         } else {
           sc.inv_l[n] = nonempty ? l : 0.0f;  // raw row sum, merged across the cluster
@@ -891,15 +905,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int wq = warp & 3;
       const int d_lane = wq * 32 + lane;
       const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-      float* po = args.part_o + (row_base * args.max_splits + s) * 512;
-      const int64_t row_stride = (int64_t)args.max_splits * 512;
+      float* po = args.part_o + (row_base * slots + slot) * 512;
+      const int64_t row_stride = (int64_t)slots * 512;
       float* staged = reinterpret_cast<float*>(smem + kOffRing);  // [64][512], ring is free
 #pragma unroll 1
       for (int ch = ewg; ch < 16; ch += 5) {
         const int j = ch >> 2, grp = ch & 3;
         float v[16];
         tmem_ld16(t_lane + kTmemO + 64 * j + 16 * grp, v);
-        if (npieces == 1) {
+        if (own) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const int nn = grp * 16 + k;
@@ -921,7 +935,111 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (npieces > 1) merge_pieces(npieces, args, smem, sc, row_base, rows_valid, s);
+  if (!own) merge_pieces(npieces, args, smem, sc, row_base, rows_valid, s);
+}
+
+// Single-launch mode, after every CTA's partial body: a grid barrier (the
+// launch is cooperative, so every CTA is resident), then the log-sum-exp
+// merge of each row's entries, spread over the grid: each 128-thread group
+// of a CTA merges one (row, 128-dim quarter) at a time, with all of a
+// thread's entry loads of a round issued before it accumulates, the split
+// weights from the entries' LSE, and sums in a fixed order (deterministic).
+// The last CTA to leave resets the two counters for the next launch.
+constexpr int kMergeGroups = kThreads / 128;
+constexpr int kMergeBatch = 32;    // entry loads in flight per thread
+
+__device__ __forceinline__ void fused_merge(const DecodeArgs& a, uint8_t* smem) {
+  Scratch& sc = *reinterpret_cast<Scratch*>(smem + kOffScratch);
+  const int tid = threadIdx.x;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();  // this CTA's partial stores, ordered by the barrier above
+    atomicAdd(a.sync, 1);
+    const uint64_t t0 = globaltimer_ns();
+    bool ok = true;
+    while (*reinterpret_cast<volatile int32_t*>(a.sync) < (int)gridDim.x) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        ok = false;
+        break;
+      }
+    }
+    __threadfence();
+    sc.merge_fail = ok ? 0 : 1;
+    if (!ok) set_error(a.dev_error, MLA_DEVERR_TIMEOUT);
+  }
+  __syncthreads();
+  if (sc.merge_fail == 0) {
+    const int grp = tid >> 7, t = tid & 127, lane = tid & 31, wid = t >> 5;
+    float* w_smem = reinterpret_cast<float*>(smem + kOffRing) + grp * 256;  // ring is free
+    float* red = reinterpret_cast<float*>(smem + kOffRing) + kMergeGroups * 256 + grp * 8;
+    const int QH = a.q_len * a.H;
+    const int rows = a.B * QH;
+    const int slots = a.max_splits * a.pieces;
+    for (int item = (int)blockIdx.x + grp * (int)gridDim.x; item < rows * 4;
+         item += kMergeGroups * (int)gridDim.x) {
+      const int row = item >> 2, d = (item & 3) * 128 + t;
+      const int bq = row / QH;
+      int S = a.num_splits[bq];
+      S = S < 1 ? 0 : (S > a.max_splits ? a.max_splits : S);
+      const int E = S * a.pieces;  // entries of this row, at most 256
+      const float* po = a.part_o + (int64_t)row * slots * 512 + d;
+      const float* pl = a.part_lse + (int64_t)row * slots;
+      float v[kMergeBatch];
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) v[j] = j < E ? __ldcg(po + (int64_t)j * 512) : 0.0f;
+      float lse[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) lse[k] = t + 128 * k < E ? __ldcg(pl + t + 128 * k) : -INFINITY;
+      float m = fmaxf(lse[0], lse[1]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      named_bar_sync(7 + grp, 128);  // red and w_smem of the previous item are no longer read
+      if (lane == 0) red[wid] = m;
+      named_bar_sync(7 + grp, 128);
+      m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      float wpart = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float w = lse[k] == -INFINITY ? 0.0f : expf(lse[k] - m);
+        if (t + 128 * k < E) w_smem[t + 128 * k] = w;
+        wpart += w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wpart += __shfl_xor_sync(0xffffffffu, wpart, o);
+      if (lane == 0) red[4 + wid] = wpart;
+      named_bar_sync(7 + grp, 128);
+      const float wsum = (red[4] + red[5]) + (red[6] + red[7]);
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int e0 = 0; e0 < E; e0 += kMergeBatch) {
+        if (e0 > 0) {
+#pragma unroll
+          for (int j = 0; j < kMergeBatch; ++j)
+            v[j] = e0 + j < E ? __ldcg(po + (int64_t)(e0 + j) * 512) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j)
+          if (e0 + j < E) acc[j & 3] = fmaf(w_smem[e0 + j], v[j], acc[j & 3]);
+      }
+      const float o = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      const bool empty = m == -INFINITY || !(wsum > 0.0f);
+      a.out[(int64_t)row * 512 + d] = __bfloat16_as_ushort(__float2bfloat16_rn(empty ? 0.0f : o / wsum));
+      if (a.out_lse != nullptr && (item & 3) == 0 && t == 0) a.out_lse[row] = empty ? -INFINITY : m + logf(wsum);
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && atomicAdd(a.sync + 1, 1) == (int)gridDim.x - 1) {
+    // every CTA has passed the barrier: leave both counters at zero
+    atomicExch(a.sync, 0);
+    atomicExch(a.sync + 1, 0);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_fp8_kernel(const DecodeArgs args, const __grid_constant__ CUtensorMap kv_map,
+                      const __grid_constant__ CUtensorMap rope_map) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  partial_body(args, &kv_map, &rope_map, smem);
+  if (args.fused) fused_merge(args, smem);
 }
 
 }  // namespace fp8k
@@ -937,6 +1055,21 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map,
   if (e != cudaSuccess) return e;
   const long long units = (long long)a.groups * a.max_splits * a.B;
   const long long ctas = a.split_from + a.pad + (units - a.split_from) * a.pieces;
+  if (a.fused) {
+    // every CTA must be resident for the grid barrier: a cooperative launch
+    // guarantees it (or fails), and the pieces need no cluster here
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(fp8k::kThreads);
+    cfg.dynamicSmemBytes = fp8k::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fp8k::decode_fp8_kernel, a, kv_map, rope_map);
+  }
   if (a.pieces == 1) {
     fp8k::decode_fp8_kernel<<<(unsigned)ctas, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map,
                                                                                          rope_map);

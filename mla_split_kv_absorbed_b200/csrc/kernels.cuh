@@ -49,6 +49,16 @@ struct DecodeArgs {
   int pad;
   int pieces;
   int inject_stall;     // test hook: leave the first load of CTA (0, 0, 0) unissued
+  // Single-launch mode (FP8, every CTA resident, cooperative launch without
+  // clusters): each piece writes its own normalised partial to entry
+  // s * pieces + piece of its rows (part_o / part_lse then hold
+  // max_splits * pieces entries per row), and after a grid barrier on
+  // sync[0] the grid merges them into out / out_lse; sync[1] counts the CTAs
+  // that have finished, and the last one resets both to zero.
+  int fused;
+  uint16_t* out;        // [rows][512] bf16
+  float* out_lse;       // [rows], may be null
+  int32_t* sync;        // two counters, zero before the launch
 };
 
 // FP8 E4M3 cache: kv_map and rope_map are 3-D tiled TMA maps over kv_pages

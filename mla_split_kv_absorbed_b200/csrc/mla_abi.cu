@@ -132,17 +132,21 @@ size_t mla_partial_workspace_bytes(int B, int q_len, int H, int max_splits) {
   return rows * 512 * sizeof(float) + rows * sizeof(float);
 }
 
-int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_pages,
-                       int kv_dtype, float kv_scale, int64_t num_pages,
-                       const int32_t* block_table, int max_pages_per_req,
-                       const int32_t* seq_lens, const int32_t* num_splits, int max_splits, int B,
-                       int q_len, int H, float softmax_scale, float* part_o, float* part_lse,
-                       int32_t* dev_error, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the partial and the single-launch entry points; fills the
+// kernel arguments (all but the output pointers) and the tensor maps.
+int setup_decode(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_pages, int kv_dtype,
+                 float kv_scale, int64_t num_pages, const int32_t* block_table,
+                 int max_pages_per_req, const int32_t* seq_lens, const int32_t* num_splits,
+                 int max_splits, int B, int q_len, int H, float softmax_scale,
+                 int32_t* dev_error, mla::DecodeArgs* a, CUtensorMap* map, CUtensorMap* rope_map) {
   if (q_nope == nullptr || q_rope == nullptr || kv_pages == nullptr || block_table == nullptr ||
-      seq_lens == nullptr || num_splits == nullptr || part_o == nullptr || part_lse == nullptr)
+      seq_lens == nullptr || num_splits == nullptr)
     return MLA_ERR_INVALID_ARG;
-  if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(kv_pages) || !aligned16(part_o))
-    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(kv_pages)) return MLA_ERR_INVALID_ARG;
   if (B <= 0 || q_len <= 0 || H <= 0 || num_pages <= 0 || max_pages_per_req <= 0 ||
       max_splits <= 0)
     return MLA_ERR_INVALID_ARG;
@@ -157,48 +161,103 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
 
   // FP8: the latent dims as 128-byte rows (128-byte swizzle) and the RoPE dims
   // as 64-byte rows (64-byte swizzle); bf16: 64-element (128-byte) rows
-  CUtensorMap map, rope_map;
-  std::memset(&map, 0, sizeof(map));
-  std::memset(&rope_map, 0, sizeof(rope_map));
+  std::memset(map, 0, sizeof(*map));
+  std::memset(rope_map, 0, sizeof(*rope_map));
   int st = kv_dtype == MLA_KV_FP8_E4M3
-               ? make_kv_map(&map, kv_pages, kv_dtype, num_pages, 128, CU_TENSOR_MAP_SWIZZLE_128B)
-               : make_kv_map(&map, kv_pages, kv_dtype, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+               ? make_kv_map(map, kv_pages, kv_dtype, num_pages, 128, CU_TENSOR_MAP_SWIZZLE_128B)
+               : make_kv_map(map, kv_pages, kv_dtype, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != MLA_OK) return st;
   if (kv_dtype == MLA_KV_FP8_E4M3) {
-    st = make_kv_map(&rope_map, kv_pages, kv_dtype, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+    st = make_kv_map(rope_map, kv_pages, kv_dtype, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_64B);
     if (st != MLA_OK) return st;
   }
 
-  mla::DecodeArgs a = {};
-  a.q_nope = q_nope;
-  a.q_rope = q_rope;
-  a.kv_pages = static_cast<const uint8_t*>(kv_pages);
-  a.block_table = block_table;
-  a.seq_lens = seq_lens;
-  a.num_splits = num_splits;
+  *a = mla::DecodeArgs{};
+  a->q_nope = q_nope;
+  a->q_rope = q_rope;
+  a->kv_pages = static_cast<const uint8_t*>(kv_pages);
+  a->block_table = block_table;
+  a->seq_lens = seq_lens;
+  a->num_splits = num_splits;
+  a->dev_error = dev_error;
+  a->num_pages = num_pages;
+  a->max_pages = max_pages_per_req;
+  a->max_splits = max_splits;
+  a->B = B;
+  a->q_len = q_len;
+  a->H = H;
+  a->qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
+  a->kv_scale = kv_scale;
+  a->inject_stall = g_inject_stall.load(std::memory_order_relaxed);
+  int32_t plan[4];
+  plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms_current_device(), plan);
+  a->groups = (q_len * H + 63) / 64;
+  a->pieces = plan[1];
+  a->split_from = plan[2];
+  a->pad = plan[3];
+  return MLA_OK;
+}
+
+constexpr size_t kFusedCounterBytes = 256;  // two int32 counters, padded
+constexpr int kFusedMaxPieces = 4;
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_pages,
+                       int kv_dtype, float kv_scale, int64_t num_pages,
+                       const int32_t* block_table, int max_pages_per_req,
+                       const int32_t* seq_lens, const int32_t* num_splits, int max_splits, int B,
+                       int q_len, int H, float softmax_scale, float* part_o, float* part_lse,
+                       int32_t* dev_error, void* stream) {
+  if (part_o == nullptr || part_lse == nullptr || !aligned16(part_o)) return MLA_ERR_INVALID_ARG;
+  mla::DecodeArgs a;
+  CUtensorMap map, rope_map;
+  const int st = setup_decode(q_nope, q_rope, kv_pages, kv_dtype, kv_scale, num_pages, block_table,
+                              max_pages_per_req, seq_lens, num_splits, max_splits, B, q_len, H,
+                              softmax_scale, dev_error, &a, &map, &rope_map);
+  if (st != MLA_OK) return st;
   a.part_o = part_o;
   a.part_lse = part_lse;
-  a.dev_error = dev_error;
-  a.num_pages = num_pages;
-  a.max_pages = max_pages_per_req;
-  a.max_splits = max_splits;
-  a.B = B;
-  a.q_len = q_len;
-  a.H = H;
-  a.qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
-  a.kv_scale = kv_scale;
-  a.inject_stall = g_inject_stall.load(std::memory_order_relaxed);
-  {
-    int32_t plan[4];
-    plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms_current_device(), plan);
-    a.groups = (q_len * H + 63) / 64;
-    a.pieces = plan[1];
-    a.split_from = plan[2];
-    a.pad = plan[3];
-  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return status_of(kv_dtype == MLA_KV_FP8_E4M3 ? mla::launch_decode_fp8(a, map, rope_map, s)
                                                : mla::launch_decode_bf16(a, map, s));
+}
+
+size_t mla_fused_workspace_bytes(int B, int q_len, int H, int max_splits) {
+  if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return 0;
+  const size_t entries = (size_t)B * q_len * H * max_splits * kFusedMaxPieces;
+  return kFusedCounterBytes + entries * 512 * sizeof(float) + entries * sizeof(float);
+}
+
+int mla_decode_fused(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_pages,
+                     int kv_dtype, float kv_scale, int64_t num_pages, const int32_t* block_table,
+                     int max_pages_per_req, const int32_t* seq_lens, const int32_t* num_splits,
+                     int max_splits, int B, int q_len, int H, float softmax_scale, void* workspace,
+                     uint16_t* out_bf16, float* out_lse, int32_t* dev_error, void* stream) {
+  if (workspace == nullptr || out_bf16 == nullptr || !aligned16(workspace))
+    return MLA_ERR_INVALID_ARG;
+  mla::DecodeArgs a;
+  CUtensorMap map, rope_map;
+  const int st = setup_decode(q_nope, q_rope, kv_pages, kv_dtype, kv_scale, num_pages, block_table,
+                              max_pages_per_req, seq_lens, num_splits, max_splits, B, q_len, H,
+                              softmax_scale, dev_error, &a, &map, &rope_map);
+  if (st != MLA_OK) return st;
+  // one launch only when every CTA of the grid is resident at once: an FP8
+  // cache and a grid that fits in one wave (every unit cut into pieces)
+  if (kv_dtype != MLA_KV_FP8_E4M3 || a.split_from != 0 || a.pieces < 2 ||
+      max_splits * a.pieces > 256)
+    return MLA_ERR_UNSUPPORTED;
+  const size_t entries = (size_t)B * q_len * H * max_splits * kFusedMaxPieces;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.fused = 1;
+  a.sync = reinterpret_cast<int32_t*>(ws);
+  a.part_o = reinterpret_cast<float*>(ws + kFusedCounterBytes);
+  a.part_lse = a.part_o + entries * 512;
+  a.out = out_bf16;
+  a.out_lse = out_lse;
+  return status_of(mla::launch_decode_fp8(a, map, rope_map, static_cast<cudaStream_t>(stream)));
 }
 
 int mla_combine(const float* part_o, const float* part_lse, const int32_t* num_splits,

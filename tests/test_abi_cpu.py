@@ -119,6 +119,24 @@ def test_rejections_without_gpu(lib):
     assert h.mla_decode_partial(*a5) == lib.MLA_ERR_INVALID_ARG
 
 
+def test_fused_workspace_and_rejections_without_gpu(lib):
+    h = lib.load()
+    null = None
+    # counters (256 bytes) + room for 4 pieces per split: O (512 fp32) and LSE per entry
+    assert h.mla_fused_workspace_bytes(1, 1, 64, 64) == 256 + 64 * 64 * 4 * 513 * 4
+    assert h.mla_fused_workspace_bytes(2, 4, 16, 8) == 256 + 2 * 4 * 16 * 8 * 4 * 513 * 4
+    assert h.mla_fused_workspace_bytes(0, 1, 64, 64) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    base = [fake, fake, fake, 0, 1.0, 10, fake, 4, fake, fake, 4, 1]
+    # null workspace / output, misaligned workspace
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, null, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, fake, null, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, mis, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    # the shared checks of mla_decode_partial apply
+    assert h.mla_decode_fused(*base, 5, 64, 1.0, fake, fake, null, null, null) == lib.MLA_ERR_UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     import mla_split_kv_absorbed_b200 as m
     monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
