@@ -6,6 +6,10 @@ step A9) on one stream, inputs resident in HBM.  The FP8 cache itself is
 produced once per run by mla_quantize_fp8 (step A1), which is timed on its
 own and reported under "quantize".
 
+When the grid fits on the GPU at once (batch 1), the same step is also timed
+through the single-launch entry point mla_decode_fused and reported under
+"single_launch".
+
 Default workload: batch 1, q_len 1, 64 heads, 128K context, FP8 E4M3 paged
 KV (page 64, shuffled block table), 64-way split.  The other four workloads
 are measured in the same run, each under its own key: "tiny" (batch 1, 16
@@ -222,6 +226,45 @@ def run_steps(w, kv, steps, warmup, flush_bytes=256 << 20):
     total = [a.elapsed_time(b) * 1e-3 for a, b in tot_ev]
     partial = [a.elapsed_time(b) * 1e-3 for a, b in par_ev]
     return total, partial
+
+
+def run_single_launch(w, kv, steps, warmup, flush_bytes=256 << 20):
+    """Per-step device times of the single-launch decode (mla_decode_fused),
+    L2 flushed before each step; None when the shape needs two kernels."""
+    import torch
+    import mla_split_kv_absorbed_b200 as m
+    stream = torch.cuda.current_stream()
+    ws_buf = m.alloc_fused_workspace(w.B, w.q_len, w.H, w.max_splits)
+    out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    out_lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
+    flush = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        m.mla_decode_fused(w.q_nope, w.q_rope, kv, w.kv_scale, w.block_table, w.seq_lens,
+                           w.num_splits, w.max_splits, w.softmax_scale, ws_buf, out, out_lse, err,
+                           stream)
+    try:
+        step()
+    except m.MlaError as e:
+        if e.status == m.MLA_ERR_UNSUPPORTED:
+            return None
+        raise
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    return [a.elapsed_time(b) * 1e-3 for a, b in evs]
 
 
 def run_e2e(w, kv, steps, warmup):
@@ -476,6 +519,7 @@ def main():
 
     e2e_t, h2d, d2h = run_e2e(w, kv, max(5, args.steps // 2), args.warmup)
     e2e_t = max_over_ranks(e2e_t, ws)
+    single = run_single_launch(w, kv, args.steps, args.warmup)
 
     extra = {}
     if not args.no_extra:
@@ -526,6 +570,12 @@ def main():
         "clocks": clk.summary(),
         "timed_wall_s": wall,
     }
+    if single is not None:
+        ts = max_over_ranks(statistics.median(single), ws)
+        line["single_launch"] = {
+            "api": "mla_decode_fused", "us_per_step": ts * 1e6,
+            "us_p10": pct(single, 0.1) * 1e6, "us_p90": pct(single, 0.9) * 1e6,
+            "kv_gbs": job_gbs(w.kv_bytes, ts, ws), "frac_of_peak": w.kv_bytes / ts / 1e9 / peak}
     if quant is not None:
         line["quantize"] = quant
     line.update(extra)

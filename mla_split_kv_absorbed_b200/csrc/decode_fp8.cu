@@ -55,9 +55,9 @@
 // Warp roles (768 threads):
 //   warp 0        TMA producer: pages -> 128-byte-swizzled 128-dim pairs
 //                 (one 8 KiB box per page and pair) in an 11-slot ring (2.75
-//                 tiles) plus a 2-slot RoPE ring (64-byte swizzle), each
-//                 tile's pages bulk-prefetched into L2 just before its loads,
-//                 its RoPE chunk loaded before its latent pairs
+//                 tiles) plus one RoPE slot (64-byte swizzle), each tile's
+//                 pages bulk-prefetched into L2 just before its loads, its
+//                 RoPE chunk loaded before its latent pairs
 //   warp 1        UMMA issuer (warp-uniform polling of readiness; the QK
 //                 MMAs whose operands have landed go before a ready PV, which
 //                 measured faster than the reverse; one elected lane issues)
@@ -87,16 +87,17 @@ constexpr int kTile = 128;          // tokens per tile (UMMA N for QK, K for PV)
 constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
 constexpr int kRingPairs = 11;      // latent pair slots: 2.75 tiles in flight
-constexpr int kRopeSlots = 2;
+constexpr int kRopeSlots = 1;      // freed by its tile's QK, refilled first for the next tile
+constexpr int kPBufs = 2;          // P buffers: the softmax of tile i+1 need not wait for PV(i)
 constexpr float kPShift = 4.0f;     // log2 of the factor carried by the softmax weights
 constexpr float kLazy = 4.75f;      // the used max moves only when exceeded by more than this
 
 constexpr int kOffRing = 0;                                  // 11 pairs
 constexpr int kOffRope = kOffRing + kRingPairs * kPair;      // 180224: 2 RoPE chunks
 constexpr int kOffQr = kOffRope + kRopeSlots * kChunk;       // 196608: Q' RoPE dims [128][64 B]
-constexpr int kOffPhi = kOffQr + kChunk;                     // 204800: P_hi [64 rows][128 B]
-constexpr int kOffPlo = kOffPhi + kChunk;                    // 212992: P_lo
-constexpr int kOffScratch = kOffPlo + kChunk;                // 221184
+constexpr int kOffP = kOffQr + kChunk;                       // buffer b: P_hi [64 rows][128 B] at
+                                                             // kOffP + 16 KiB b, P_lo 8 KiB after it
+constexpr int kOffScratch = kOffP + kPBufs * 2 * kChunk;
 constexpr int kSmemBytes = 232448;                           // 227 KiB
 
 constexpr uint32_t kTmemO = 0;      // O^T block j at 64 j
@@ -104,20 +105,21 @@ constexpr uint32_t kTmemQ = 256;    // Q' latent dims: K step k at 256 + 8 k
 constexpr uint32_t kTmemS = 384;    // S' [128 rows][128 tokens]
 
 // barrier indices
-constexpr int kBarFull = 0;                      // 11
-constexpr int kBarEmpty = kBarFull + kRingPairs;  // 11
-constexpr int kBarRopeFull = 22;   // 2
-constexpr int kBarRopeEmpty = 24;  // 2
-constexpr int kBarSFull = 26;
-constexpr int kBarSEmpty = 27;     // one arrival per softmax warp
-constexpr int kBarPFull = 28;      // one arrival per softmax warp
-constexpr int kBarPEmpty = 29;
-constexpr int kBarOReady = 30;     // 2: per tile parity (the rescale loop may run a tile ahead)
-constexpr int kBarPvDone = 32;
-constexpr int kBarQReady = 33;     // one arrival per softmax warp
-constexpr int kBarAlphaFull = 34;  // 2: per tile parity, one arrival per lane quadrant
-constexpr int kBarDrain = 36;
-constexpr int kNumBars = 37;
+constexpr int kBarFull = 0;                           // kRingPairs
+constexpr int kBarEmpty = kBarFull + kRingPairs;      // kRingPairs
+constexpr int kBarRopeFull = kBarEmpty + kRingPairs;  // kRopeSlots
+constexpr int kBarRopeEmpty = kBarRopeFull + kRopeSlots;
+constexpr int kBarSFull = kBarRopeEmpty + kRopeSlots;
+constexpr int kBarSEmpty = kBarSFull + 1;      // one arrival per softmax warp
+constexpr int kBarPFull = kBarSEmpty + 1;      // kPBufs, one arrival per softmax warp
+constexpr int kBarPEmpty = kBarPFull + kPBufs;  // kPBufs
+constexpr int kBarOReady = kBarPEmpty + kPBufs;  // 2: per tile parity
+constexpr int kBarPvDone = kBarOReady + 2;
+constexpr int kBarQReady = kBarPvDone + 1;
+constexpr int kBarAlphaFull = kBarQReady + 1;  // 2: per tile parity, one arrival per lane quadrant
+constexpr int kBarDrain = kBarAlphaFull + 2;
+constexpr int kBarPvAll = kBarDrain + 1;
+constexpr int kNumBars = kBarPvAll + 1;
 
 struct Scratch {
   uint64_t bars[40];
@@ -208,7 +210,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs& args, uint8_t* sm
   const uint32_t rank = cluster_ctarank();
   cluster_sync_all();  // every piece's O, m and l are staged
   const int n0 = (int)rank * kRowsPer;
-  float* wgt = reinterpret_cast<float*>(smem + kOffPhi);  // [P][64] piece weights (P buffers are free)
+  float* wgt = reinterpret_cast<float*>(smem + kOffP);  // [P][64] piece weights (P buffers are free)
   if (tid < kRowsPer) {
     const int n = n0 + tid;
     float mk[P], lk[P];
@@ -391,8 +393,11 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
     }
     mbar_init(&sc.bars[kBarSFull], 1);
     mbar_init(&sc.bars[kBarSEmpty], kSoftWarps);
-    mbar_init(&sc.bars[kBarPFull], kSoftWarps);
-    mbar_init(&sc.bars[kBarPEmpty], 1);
+    for (int i = 0; i < kPBufs; ++i) {
+      mbar_init(&sc.bars[kBarPFull + i], kSoftWarps);
+      mbar_init(&sc.bars[kBarPEmpty + i], 1);
+    }
+    mbar_init(&sc.bars[kBarPvAll], 1);
     for (int i = 0; i < 2; ++i) mbar_init(&sc.bars[kBarOReady + i], 4);
     mbar_init(&sc.bars[kBarPvDone], 1);
     mbar_init(&sc.bars[kBarQReady], kSoftWarps);
@@ -454,7 +459,8 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
     int last_parity[kRingPairs];
     bool armed[kRingPairs];
     for (int i = 0; i < kRingPairs; ++i) armed[i] = false;
-    int rope_last[kRopeSlots] = {-1, -1};
+    int rope_last[kRopeSlots];
+    for (int q = 0; q < kRopeSlots; ++q) rope_last[q] = -1;
     bool ok = true;
     int u = 0;  // load number of the next latent pair
     for (int i = 0; i < T && ok; ++i) {
@@ -532,8 +538,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
     const uint64_t dRope = smem_desc(smem_u32(smem + kOffRope), 16, 512, 4);
     const uint64_t dQr = smem_desc(smem_u32(smem + kOffQr), 16, 512, 4);
     const uint64_t dRingMN = smem_desc(smem_u32(smem + kOffRing), kPair, 1024, 2);
-    const uint64_t dPhi = smem_desc(smem_u32(smem + kOffPhi), 16, 1024, 2);
-    const uint64_t dPlo = smem_desc(smem_u32(smem + kOffPlo), 16, 1024, 2);
+    const uint64_t dP = smem_desc(smem_u32(smem + kOffP), 16, 1024, 2);  // buffer 0, P_hi
     const uint32_t d_s = tmem + kTmemS;
     auto ready = [&](int bar, int parity) {
       return __any_sync(0xffffffffu, mbar_test_wait(&bars[bar], parity));
@@ -588,8 +593,10 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
         }
       }
       // ---------------- O^T += V(np)^T . (P_hi + P_lo), after any QK that was ready
-      if (np < nq && ready(kBarPFull, np & 1) && ready(kBarOReady + (np & 1), (np >> 1) & 1)) {
+      if (np < nq && ready(kBarPFull + (np & 1), (np >> 1) & 1) &&
+          ready(kBarOReady + (np & 1), (np >> 1) & 1)) {
         tc_fence_after();
+        const uint64_t dPhi = desc_at(dP, (np & 1) * 2 * kChunk), dPlo = desc_at(dPhi, kChunk);
         // block by block, so each latent pair can be refilled as soon as its
         // block is done
 #pragma unroll
@@ -605,8 +612,9 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
           // latent pair j of this tile is free once its block's MMAs complete
           umma_commit_elect(&bars[kBarEmpty + slot]);
         }
-        umma_commit_elect(&bars[kBarPEmpty]);
+        umma_commit_elect(&bars[kBarPEmpty + (np & 1)]);
         umma_commit_elect(&bars[kBarPvDone]);
+        if (np == T - 1) umma_commit_elect(&bars[kBarPvAll]);
         ++np;
         progress = true;
       }
@@ -780,6 +788,11 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
           m_run = tm;
         }
       }
+      // P buffer i % 2 free: PV of tile i - 2 done.  Waited for before this
+      // tile's alpha goes out: PV(i - 2) waited for the rescale of tile i - 2,
+      // so that alpha slot has been read, and the PV-done count the rescale
+      // warps test is at least i - 1.
+      if (i >= kPBufs) bad |= !mbar_wait(&bars[kBarPEmpty + (i & 1)], ((i >> 1) - 1) & 1, abort_flag);
       // the rescale warps learn, per tile, which rows moved and by how much
       if (c == 0) {
         const uint32_t mask = __ballot_sync(0xffffffffu, moved && part == 0);
@@ -799,11 +812,9 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
       l_run = fmaf(l_run, alpha, psum);
       uint4 phi, plo;
       split16(pv, phi, plo);
-      // P buffer (and the V rows cleared below) free: PV of the previous tile done
-      if (i >= 1) bad |= !mbar_wait(&bars[kBarPEmpty], (i - 1) & 1, abort_flag);
-      const uint32_t p_off = sw128(n, 32 * c + 16 * part);
-      *reinterpret_cast<uint4*>(smem + kOffPhi + p_off) = phi;
-      *reinterpret_cast<uint4*>(smem + kOffPlo + p_off) = plo;
+      const uint32_t p_off = kOffP + (i & 1) * 2 * kChunk + sw128(n, 32 * c + 16 * part);
+      *reinterpret_cast<uint4*>(smem + p_off) = phi;
+      *reinterpret_cast<uint4*>(smem + p_off + kChunk) = plo;
       if (t0 + i * kTile + kTile > t1) {
         // token rows past the visible range: clear their V bytes so that
         // 0 * garbage cannot be NaN (thread: token row tid_s & 127, pair tid_s >> 7)
@@ -817,7 +828,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarPFull]);
+      if (lane == 0) mbar_arrive(&bars[kBarPFull + (i & 1)]);
     }
     // ---- row sums: reduce l over the 8 threads of row n, in a fixed order
     {
@@ -844,7 +855,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
     // ============================================================ O^T rescale between tiles
     // The O-ready barriers are per tile parity because this loop may run one
     // tile ahead of the PV issue, but never two: the softmax of tile i + 2
-    // needs the P buffer that PV(i) frees, and so its max and alpha.
+    // sends its alpha only after PV(i), which waited for this loop's tile i.
     const int wq = warp & 3;            // thread = latent dim wq * 32 + lane of a block
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     bool ok = true;
@@ -884,13 +895,9 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarOReady + (i & 1)]);
     }
-    // This loop may have run a tile ahead of PV, so the barrier can still be
-    // one phase short of tile T-2: wait for that phase first, or the parity
-    // test for T-1 would match the older phase T-3.
-    if (ok && wq == 0 && lane == 0) {
-      if (T >= 2) mbar_wait(&bars[kBarPvDone], (T - 2) & 1, abort_flag);
-      mbar_wait(&bars[kBarPvDone], (T - 1) & 1, abort_flag);
-    }
+    // every PV complete (a barrier of its own: the PV-done count may be one
+    // or two tiles behind here, which one parity test cannot tell apart)
+    if (ok && wq == 0 && lane == 0) mbar_wait(&bars[kBarPvAll], 0, abort_flag);
     named_bar_sync(5, 128);
     tc_fence_before();
     named_bar_sync(6, kSoftThreads + 128);  // inv_l ready, every PV complete
