@@ -233,6 +233,8 @@ def run_single_launch(w, kv, steps, warmup, flush_bytes=256 << 20):
     L2 flushed before each step; None when the shape needs two kernels."""
     import torch
     import mla_split_kv_absorbed_b200 as m
+    if w.spec.kv_dtype != "fp8":
+        return None
     stream = torch.cuda.current_stream()
     ws_buf = m.alloc_fused_workspace(w.B, w.q_len, w.H, w.max_splits)
     out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
