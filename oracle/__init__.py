@@ -63,6 +63,8 @@ def _load():
                                            ctypes.POINTER(i64)]
         lib.oracle_mla_partials_rows.argtypes = [P, P, P, i32, f32, P, i32, P, P, i32, i32,
                                                  i32, i32, f32, P, i64, P, P]
+        lib.oracle_mla_partials_rows_q8.argtypes = [P, f32, P, i32, f32, P, i32, P, P, i32, i32,
+                                                    i32, i32, f32, P, i64, P, P]
         lib.oracle_combine.argtypes = [P, P, P, i32, i64, P, P]
         lib.oracle_num_threads.restype = i32
         lib.oracle_rope_f64.argtypes = [P, i64, ctypes.c_double, P]
@@ -160,6 +162,27 @@ def partials_rows(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num
                                  _ptr(bt), bt.shape[1], _ptr(sl), _ptr(ns), int(max_splits), B,
                                  q_len, H, float(softmax_scale), _ptr(rows), rows.size, _ptr(o),
                                  _ptr(lse))
+    return o, lse
+
+
+def partials_rows_q8(q8, q_scale, kv_pages, kv_scale, block_table, seq_lens, num_splits,
+                     max_splits, q_len, H, softmax_scale, rows):
+    """partials_rows with an FP8 query: q8 uint8 E4M3 codes [B][q_len][H][576]
+    (latent then RoPE dims) of value code * q_scale."""
+    lib = _load()
+    kv_dtype, kv = _kv_args(kv_pages)
+    q = np.ascontiguousarray(q8, dtype=np.uint8)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    ns = np.ascontiguousarray(num_splits, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    B = sl.shape[0]
+    o = np.zeros((rows.size, max_splits, D_LATENT), dtype=np.float64)
+    lse = np.zeros((rows.size, max_splits), dtype=np.float64)
+    lib.oracle_mla_partials_rows_q8(_ptr(q), float(np.float32(q_scale)), _ptr(kv), kv_dtype,
+                                    float(kv_scale), _ptr(bt), bt.shape[1], _ptr(sl), _ptr(ns),
+                                    int(max_splits), B, q_len, H, float(softmax_scale),
+                                    _ptr(rows), rows.size, _ptr(o), _ptr(lse))
     return o, lse
 
 

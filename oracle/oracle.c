@@ -143,7 +143,7 @@ static int64_t page_of(const int32_t* block_table, int max_pages, int b, int64_t
  *   m = max s,  O = sum e^{s_t-m} v_t / sum e^{s_t-m},  LSE = m + ln sum e^{s_t-m}
  * with v_t the first 512 dims of token t's row.  An empty range gives O = 0,
  * LSE = -inf.  Two passes over the tokens: scores and max, then weights. */
-static void attend_range(const uint16_t* qn, const uint16_t* qr, const void* kv_pages,
+static void attend_range(const double* q, const void* kv_pages,
                          int kv_dtype, double kv_scale, const int32_t* block_table,
                          int max_pages, int b, int64_t t0, int64_t t1,
                          double softmax_scale, double* o, double* lse, double* s_buf) {
@@ -152,9 +152,6 @@ static void attend_range(const uint16_t* qn, const uint16_t* qr, const void* kv_
     *lse = -INFINITY;
     return;
   }
-  double q[D_ROW];
-  for (int d = 0; d < D_LATENT; ++d) q[d] = (double)bf16_to_f32(qn[d]);
-  for (int d = 0; d < D_ROPE; ++d) q[D_LATENT + d] = (double)bf16_to_f32(qr[d]);
 
   double m = -INFINITY;
   for (int64_t t = t0; t < t1; ++t) {
@@ -178,6 +175,12 @@ static void attend_range(const uint16_t* qn, const uint16_t* qr, const void* kv_
   }
   for (int d = 0; d < D_LATENT; ++d) o[d] /= l;
   *lse = m + log(l);
+}
+
+/* A bf16 query row (q_nope then q_rope) as 576 fp64 values. */
+static void q_from_bf16(const uint16_t* qn, const uint16_t* qr, double* q) {
+  for (int d = 0; d < D_LATENT; ++d) q[d] = (double)bf16_to_f32(qn[d]);
+  for (int d = 0; d < D_ROPE; ++d) q[D_LATENT + d] = (double)bf16_to_f32(qr[d]);
 }
 
 /* Causal visible length of query position q of request b (seq_len includes
@@ -208,8 +211,9 @@ void oracle_mla_decode_rows(const uint16_t* q_nope, const uint16_t* q_rope,
       int q = (int)((r / H) % q_len);
       int b = (int)(r / ((int64_t)H * q_len));
       int64_t vis = visible_len(seq_lens[b], q_len, q);
-      attend_range(q_nope + r * D_LATENT, q_rope + r * D_ROPE, kv_pages, kv_dtype,
-                   (double)kv_scale, block_table, max_pages, b, 0, vis,
+      double qv[D_ROW];
+      q_from_bf16(q_nope + r * D_LATENT, q_rope + r * D_ROPE, qv);
+      attend_range(qv, kv_pages, kv_dtype, (double)kv_scale, block_table, max_pages, b, 0, vis,
                    (double)softmax_scale, out_o + i * D_LATENT, out_lse + i, s_buf);
     }
     free(s_buf);
@@ -266,9 +270,50 @@ void oracle_mla_partials_rows(const uint16_t* q_nope, const uint16_t* q_rope,
         if (s < num_splits[b])
           oracle_split_range(seq_lens[b], num_splits[b], s,
                              visible_len(seq_lens[b], q_len, q), &t0, &t1);
-        attend_range(q_nope + r * D_LATENT, q_rope + r * D_ROPE, kv_pages, kv_dtype,
-                     (double)kv_scale, block_table, max_pages, b, t0, t1,
-                     (double)softmax_scale, o, lse, s_buf);
+        double qv[D_ROW];
+        q_from_bf16(q_nope + r * D_LATENT, q_rope + r * D_ROPE, qv);
+        attend_range(qv, kv_pages, kv_dtype, (double)kv_scale, block_table, max_pages, b, t0,
+                     t1, (double)softmax_scale, o, lse, s_buf);
+      }
+    }
+    free(s_buf);
+  }
+}
+
+/* Per-split partials with an FP8 query (page 1, bullet "原生 FP8 转换": the
+ * prep converts Q to FP8 as well as KV).  Query row r is the 576 E4M3 codes
+ * q8[r*576 .. r*576+575] (512 latent dims, then 64 RoPE dims), whose values
+ * are e4m3(code) * q_scale with one per-tensor scale; splits, causality and
+ * the output layout are those of oracle_mla_partials_rows. */
+void oracle_mla_partials_rows_q8(const uint8_t* q8, float q_scale, const void* kv_pages,
+                                 int kv_dtype, float kv_scale, const int32_t* block_table,
+                                 int max_pages, const int32_t* seq_lens,
+                                 const int32_t* num_splits, int max_splits, int B, int q_len,
+                                 int H, float softmax_scale, const int64_t* rows,
+                                 int64_t n_rows, double* out_o, double* out_lse) {
+  init_tables();
+  int64_t max_len = 0;
+  for (int b = 0; b < B; ++b)
+    if (seq_lens[b] > max_len) max_len = seq_lens[b];
+#pragma omp parallel
+  {
+    double* s_buf = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+#pragma omp for schedule(dynamic, 1) collapse(2)
+    for (int64_t i = 0; i < n_rows; ++i) {
+      for (int s = 0; s < max_splits; ++s) {
+        int64_t r = rows[i];
+        int q = (int)((r / H) % q_len);
+        int b = (int)(r / ((int64_t)H * q_len));
+        double* o = out_o + (i * max_splits + s) * D_LATENT;
+        double* lse = out_lse + i * max_splits + s;
+        int64_t t0 = 0, t1 = 0;
+        if (s < num_splits[b])
+          oracle_split_range(seq_lens[b], num_splits[b], s,
+                             visible_len(seq_lens[b], q_len, q), &t0, &t1);
+        double qv[D_ROW];
+        for (int d = 0; d < D_ROW; ++d) qv[d] = g_e4m3[q8[r * D_ROW + d]] * (double)q_scale;
+        attend_range(qv, kv_pages, kv_dtype, (double)kv_scale, block_table, max_pages, b, t0,
+                     t1, (double)softmax_scale, o, lse, s_buf);
       }
     }
     free(s_buf);

@@ -437,3 +437,40 @@ def test_append_skips_out_of_range_tokens(oracle_lib):
     bt2[0, 0] = num_pages + 5  # page id outside the pool
     kv2 = np.zeros_like(kv)
     assert oracle_lib.append_kv(c, r, oracle_lib.rope_table(256), bt2, sl, 2, 1.0, kv2) == 2
+
+
+def test_fp8_query_partials_equal_the_bf16_path_on_the_dequantised_query(oracle_lib):
+    # The FP8-query entry point reads 576 E4M3 codes per row with one scale.
+    # With a power-of-two scale the dequantised query is exactly bf16, so the
+    # bf16 entry point (pinned against dense NumPy above) on those values must
+    # give the same partials; with one split it must match dense NumPy too.
+    rng = np.random.default_rng(11)
+    c = _case(rng, 2, 2, 3, [130, 70], fp8=True)
+    q_scale = 0.0625
+    qbits = np.concatenate([c["q_nope"], c["q_rope"]], axis=-1)       # [B][q][H][576] bf16
+    q8 = oracle_lib.quantize(qbits, float(np.float32(1.0) / np.float32(q_scale)))
+    qv = npr.e4m3_values(q8) * q_scale
+    assert np.all(np.isfinite(qv))
+    vbits = (qv.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(npr.bf16_bits_to_f64(vbits), qv)
+    rows = _all_rows(c)
+    ns = np.array([3, 2], dtype=np.int32)
+    args = (c["kv_pages"], c["kv_scale"], c["block_table"], c["seq_lens"], ns, 3, c["q_len"], c["H"],
+            c["softmax_scale"], rows)
+    o8, l8 = oracle_lib.partials_rows_q8(q8, q_scale, *args)
+    ob, lb = oracle_lib.partials_rows(np.ascontiguousarray(vbits[..., :512]),
+                                      np.ascontiguousarray(vbits[..., 512:]), *args)
+    np.testing.assert_allclose(o8, ob, rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(np.isneginf(l8), np.isneginf(lb))
+    fin = np.isfinite(lb)
+    np.testing.assert_allclose(l8[fin], lb[fin], rtol=1e-13)
+    # one split: the unsplit decode, against dense NumPy on the dequantised query
+    o1, l1 = oracle_lib.partials_rows_q8(q8, q_scale, c["kv_pages"], c["kv_scale"], c["block_table"],
+                                         c["seq_lens"], np.ones(2, np.int32), 1, c["q_len"], c["H"],
+                                         c["softmax_scale"], rows)
+    c2 = dict(c)
+    c2["q_nope"] = np.ascontiguousarray(vbits[..., :512])
+    c2["q_rope"] = np.ascontiguousarray(vbits[..., 512:])
+    O, LSE = npr.attend(**c2)
+    np.testing.assert_allclose(o1[:, 0], O.reshape(-1, 512), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(l1[:, 0], LSE.reshape(-1), rtol=1e-11, atol=1e-12)
