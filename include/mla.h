@@ -127,6 +127,26 @@ MLA_API int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope,
                        int32_t* dev_error, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Steps A2-A8 with an FP8 query (article bullet "原生 FP8 转换": the prep
+ * converts Q to FP8 as well as KV).  An option beside mla_decode_partial, not
+ * its replacement: the query itself is then quantised, which the bf16-query
+ * entry point avoids (it splits Q into two exact FP8 terms), so results
+ * differ from it by the query's rounding.  The MMAs take the same time.
+ * q8 [B][q_len][H][576] E4M3 codes (the 512 latent dims, then the 64 RoPE
+ * dims; e.g. from mla_quantize_fp8 of the concatenated bf16 query), 16-byte
+ * aligned; the value of a code is e4m3(code) * q_scale (q_scale > 0, finite).
+ * kv_pages must be FP8 E4M3.  Every other argument, the outputs and the
+ * error behaviour are those of mla_decode_partial; merge with mla_combine.
+ * ------------------------------------------------------------------------- */
+MLA_API int mla_decode_partial_q8(const uint8_t* q8, float q_scale, const void* kv_pages,
+                                  float kv_scale, int64_t num_pages,
+                                  const int32_t* block_table, int max_pages_per_req,
+                                  const int32_t* seq_lens, const int32_t* num_splits,
+                                  int max_splits, int B, int q_len, int H, float softmax_scale,
+                                  float* part_o, float* part_lse, int32_t* dev_error,
+                                  void* stream);
+
+/* ---------------------------------------------------------------------------
  * Step A9: the second kernel, LSE merge of the partials (same bullet): per row
  *   M = max_s LSE_s, w_s = e^{LSE_s - M},
  *   O = sum_s w_s O_s / sum_s w_s (rounded to bf16, nearest-even),

@@ -11,6 +11,8 @@ Entry points (same names as the C ABI):
 * ``mla_quantize_fp8(x_bf16, y_u8, inv_scale)`` — step A1, saturating E4M3.
 * ``mla_decode_partial(...)`` — steps A2-A8, per-split partial O and LSE.
 * ``mla_combine(...)`` — step A9, log-sum-exp merge into bf16 O and fp32 LSE.
+* ``mla_decode_partial_q8(...)`` — steps A2-A8 with an FP8 query (E4M3 codes and
+  one scale), an option beside the exact two-term bf16 query.
 * ``mla_decode_fused(...)`` — steps A2-A9 in one cooperative launch (FP8, grids
   that fit on the GPU at once, e.g. batch 1); ``mla_fused_workspace_bytes`` and
   ``alloc_fused_workspace`` size and zero its workspace.
@@ -49,7 +51,8 @@ EXPORTS = ("mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partia
            "mla_combine", "mla_choose_splits", "mla_device_error_status", "mla_status_string",
            "mla_decode_noalloc", "mla_partial_grid", "mla_debug_inject_stall",
            "mla_append_kv_fp8", "mla_rope_cos_sin_table", "mla_combine_f32",
-           "mla_merge_rank_partials", "mla_fused_workspace_bytes", "mla_decode_fused")
+           "mla_merge_rank_partials", "mla_fused_workspace_bytes", "mla_decode_fused",
+           "mla_decode_partial_q8")
 
 
 class MlaError(RuntimeError):
@@ -107,6 +110,9 @@ def _load_lib():
     lib.mla_decode_fused.argtypes = [P, P, P, i32, f32, i64, P, i32, P, P, i32, i32, i32, i32,
                                      f32, P, P, P, P, P]
     lib.mla_decode_fused.restype = i32
+    lib.mla_decode_partial_q8.argtypes = [P, f32, P, f32, i64, P, i32, P, P, i32, i32, i32, i32,
+                                          f32, P, P, P, P]
+    lib.mla_decode_partial_q8.restype = i32
     return lib
 
 
@@ -228,6 +234,29 @@ def mla_decode_fused(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, 
         None if out_lse is None else _dev(out_lse, "out_lse", torch.float32),
         None if dev_error is None else _dev(dev_error, "dev_error", torch.int32), _stream(stream)))
     return out
+
+
+def mla_decode_partial_q8(q8, q_scale, kv_pages, kv_scale, block_table, seq_lens, num_splits,
+                          max_splits, softmax_scale, part_o, part_lse, dev_error=None,
+                          stream=None):
+    """Split-KV partial attention with an FP8 query: q8 uint8 E4M3 codes
+    [B][q_len][H][576] (latent then RoPE dims) of value code * q_scale."""
+    B, q_len, H, dq = q8.shape
+    if dq != 576 or q8.dtype != torch.uint8:
+        raise ValueError("q8 must be uint8 [B][q_len][H][576]")
+    if kv_pages.dtype != torch.uint8 or kv_pages.dim() != 3 or tuple(kv_pages.shape[1:]) != (64, 576):
+        raise ValueError("kv_pages must be uint8 (E4M3 codes) [num_pages][64][576]")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B][max_pages]")
+    if part_o.numel() != B * q_len * H * max_splits * 512 or part_lse.numel() != B * q_len * H * max_splits:
+        raise ValueError("partial buffers have the wrong size")
+    _check("mla_decode_partial_q8", _lib.mla_decode_partial_q8(
+        _dev(q8, "q8", torch.uint8), float(q_scale), _dev(kv_pages, "kv_pages"), float(kv_scale),
+        kv_pages.shape[0], _dev(block_table, "block_table", torch.int32), block_table.shape[1],
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(num_splits, "num_splits", torch.int32),
+        int(max_splits), B, q_len, H, float(softmax_scale),
+        _dev(part_o, "part_o", torch.float32), _dev(part_lse, "part_lse", torch.float32),
+        None if dev_error is None else _dev(dev_error, "dev_error", torch.int32), _stream(stream)))
 
 
 def mla_combine(part_o, part_lse, num_splits, max_splits, out, out_lse=None, stream=None):

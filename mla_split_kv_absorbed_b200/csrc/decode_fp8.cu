@@ -645,7 +645,41 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
     const bool valid = n < rows_valid;
     const int bar_id = 1 + qd;         // the four warps of this quadrant
     float c_head;                      // softmax_scale * kv_scale * log2(e) * 2^-e
-    {
+    if (args.q8 != nullptr) {
+      // ---- FP8 query: row n's slice c is its own E4M3 codes, used as they
+      // are (a single term: the hi lanes hold the codes, the lo lanes zeros),
+      // with the per-tensor scale folded into the score factor.
+      const uint8_t* qrow = args.q8 + (row_base + n) * 576;
+      const bool mine = valid && part == 0;
+      uint32_t w[32];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint4 x = mine ? *reinterpret_cast<const uint4*>(qrow + 128 * c + 16 * k)
+                             : make_uint4(0, 0, 0, 0);
+        w[4 * k] = x.x;
+        w[4 * k + 1] = x.y;
+        w[4 * k + 2] = x.z;
+        w[4 * k + 3] = x.w;
+      }
+      const uint4 r8 = mine ? *reinterpret_cast<const uint4*>(qrow + 512 + 16 * c)
+                            : make_uint4(0, 0, 0, 0);
+      c_head = valid ? args.qk_scale_log2 * args.q_scale : 0.0f;
+      const uint32_t t_q = tmem + ((uint32_t)(32 * qd) << 16) + kTmemQ + 32 * c;
+      float first[16], second[16];  // slice dims [0, 64) and [64, 128)
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        first[k] = __uint_as_float(w[k]);
+        second[k] = __uint_as_float(w[16 + k]);
+      }
+      tmem_st16(t_q, first);
+      tmem_st16(t_q + 16, second);
+      *reinterpret_cast<uint4*>(smem + kOffQr + sw64(32 * qd + lane, 16 * c)) = r8;
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarQReady]);
+    } else {
       // ---- Q -> Q' = [Q_hi ; Q_lo] with a power-of-two scale per query row.
       // Row n's slice c is latent dims [128c, 128c+128) and RoPE dims
       // [16c, 16c+16); the two lanes of the row (l and l ^ 16) each load one

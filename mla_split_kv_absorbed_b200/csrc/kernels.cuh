@@ -49,6 +49,11 @@ struct DecodeArgs {
   int pad;
   int pieces;
   int inject_stall;     // test hook: leave the first load of CTA (0, 0, 0) unissued
+  // FP8 query (FP8 kernel only): when q8 is set, query row r is the 576 E4M3
+  // codes q8[576 r ..] (latent then RoPE dims) of value code * q_scale, and
+  // q_nope / q_rope are not read.
+  const uint8_t* q8;
+  float q_scale;
   // Single-launch mode (FP8, every CTA resident, cooperative launch without
   // clusters): each piece writes its own normalised partial to entry
   // s * pieces + piece of its rows (part_o / part_lse then hold

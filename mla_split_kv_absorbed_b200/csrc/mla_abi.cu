@@ -225,6 +225,30 @@ int mla_decode_partial(const uint16_t* q_nope, const uint16_t* q_rope, const voi
                                                : mla::launch_decode_bf16(a, map, s));
 }
 
+int mla_decode_partial_q8(const uint8_t* q8, float q_scale, const void* kv_pages, float kv_scale,
+                          int64_t num_pages, const int32_t* block_table, int max_pages_per_req,
+                          const int32_t* seq_lens, const int32_t* num_splits, int max_splits,
+                          int B, int q_len, int H, float softmax_scale, float* part_o,
+                          float* part_lse, int32_t* dev_error, void* stream) {
+  if (q8 == nullptr || !aligned16(q8) || part_o == nullptr || part_lse == nullptr ||
+      !aligned16(part_o))
+    return MLA_ERR_INVALID_ARG;
+  if (!(q_scale > 0.0f) || !(q_scale < INFINITY)) return MLA_ERR_INVALID_ARG;
+  mla::DecodeArgs a;
+  CUtensorMap map, rope_map;
+  // the query pointers of the bf16 form are not read in this mode: q8 stands in
+  const uint16_t* qq = reinterpret_cast<const uint16_t*>(q8);
+  const int st = setup_decode(qq, qq, kv_pages, MLA_KV_FP8_E4M3, kv_scale, num_pages, block_table,
+                              max_pages_per_req, seq_lens, num_splits, max_splits, B, q_len, H,
+                              softmax_scale, dev_error, &a, &map, &rope_map);
+  if (st != MLA_OK) return st;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.q8 = q8;
+  a.q_scale = q_scale;
+  return status_of(mla::launch_decode_fp8(a, map, rope_map, static_cast<cudaStream_t>(stream)));
+}
+
 size_t mla_fused_workspace_bytes(int B, int q_len, int H, int max_splits) {
   if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return 0;
   const size_t entries = (size_t)B * q_len * H * max_splits * kFusedMaxPieces;

@@ -137,6 +137,20 @@ def test_fused_workspace_and_rejections_without_gpu(lib):
     assert h.mla_decode_fused(*base, 5, 64, 1.0, fake, fake, null, null, null) == lib.MLA_ERR_UNSUPPORTED
 
 
+def test_q8_rejections_without_gpu(lib):
+    h = lib.load()
+    null = None
+    fake = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    rest = [fake, 1.0, 10, fake, 4, fake, fake, 4, 1, 1, 64, 1.0, fake, fake, null, null]
+    assert h.mla_decode_partial_q8(null, 1.0, *rest) == lib.MLA_ERR_INVALID_ARG      # no query
+    assert h.mla_decode_partial_q8(mis, 1.0, *rest) == lib.MLA_ERR_INVALID_ARG       # misaligned
+    assert h.mla_decode_partial_q8(fake, 0.0, *rest) == lib.MLA_ERR_INVALID_ARG      # q_scale <= 0
+    assert h.mla_decode_partial_q8(fake, float("inf"), *rest) == lib.MLA_ERR_INVALID_ARG
+    bad_rows = [fake, 1.0, 10, fake, 4, fake, fake, 4, 1, 5, 64, 1.0, fake, fake, null, null]
+    assert h.mla_decode_partial_q8(fake, 1.0, *bad_rows) == lib.MLA_ERR_UNSUPPORTED  # q_len 5
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     import mla_split_kv_absorbed_b200 as m
     monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
