@@ -57,3 +57,46 @@ def test_stalled_load_times_out_and_context_survives(case):
     o_ref, l_ref = oracle_rows(c, rows)
     assert_attention_close(out.float().cpu().numpy().reshape(-1, 512),
                            lse.cpu().numpy().reshape(-1), o_ref, l_ref, what="after timeout")
+
+
+def test_single_launch_with_a_stalled_piece_reports_and_resets_its_counters():
+    # The single-launch path: CTA 0's stalled load runs its waits out, the
+    # other CTAs wait for it at the grid barrier (also bounded), the timeout
+    # is reported, the workspace counters are back at zero, and the next
+    # single launch on the same workspace is correct.
+    import mla_split_kv_absorbed_b200 as m
+    c = make_case("b1_128k_fp8", seq_lens=[8192], splits=4)
+    w = c.w
+    ws = m.alloc_fused_workspace(w.B, w.q_len, w.H, w.max_splits)
+    out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def fused():
+        m.mla_decode_fused(c.dev["q_nope"], c.dev["q_rope"], c.kv_dev, w.kv_scale,
+                           c.dev["block_table"], c.dev["seq_lens"], c.dev["num_splits"],
+                           w.max_splits, w.softmax_scale, ws, out, lse, err)
+
+    torch.cuda.synchronize()
+    prev = m.mla_debug_inject_stall(True)
+    try:
+        t0 = time.perf_counter()
+        fused()
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        m.mla_debug_inject_stall(prev)
+    word = int(err.item())
+    print(f"[failure] single launch: error word {word:#x} after {elapsed:.2f} s")
+    assert word & m.DEVERR_TIMEOUT, f"timeout not reported (error word {word:#x})"
+    assert elapsed < 30.0
+    assert torch.count_nonzero(ws[:8]).item() == 0
+
+    err.zero_()
+    fused()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rows = np.arange(w.B * w.q_len * w.H)
+    o_ref, l_ref = oracle_rows(c, rows)
+    assert_attention_close(out.float().cpu().numpy().reshape(-1, 512),
+                           lse.cpu().numpy().reshape(-1), o_ref, l_ref, what="single launch after timeout")
