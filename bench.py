@@ -1,24 +1,28 @@
 """Benchmark: absorbed-MLA split-KV decode step on B200.
 
-A step is one pass of the decode hot path over one batch: mla_decode_partial
-(split-KV partial attention, steps A2-A8) followed by mla_combine (LSE merge,
-step A9) on one stream, inputs resident in HBM.  The FP8 cache itself is
-produced once per run by mla_quantize_fp8 (step A1), which is timed on its
-own and reported under "quantize".
+A step is one pass of the decode hot path (steps A2-A9) over one batch, inputs
+resident in HBM, through the call a user makes for that shape:
 
-When the grid fits on the GPU at once (batch 1), the same step is also timed
-through the single-launch entry point mla_decode_fused and reported under
-"single_launch".
+* FP8 cache and at most one (64-row group, request) pair per SM: the single
+  launch mla_decode_fused.  It cuts every request into S equal page ranges, S
+  as large as one wave of CTAs allows (148 at batch 1, 9 at batch 16 on 148
+  SMs), and merges the partials after a grid barrier in the same kernel.
+* otherwise mla_decode_partial followed by mla_combine, with the workload's
+  own split count.
+
+The two-kernel step with the workload's split count (64 at batch 1, 32 at
+batch 16) is timed as well for every workload and reported under
+"two_kernel".  The FP8 cache itself is produced once per run by
+mla_quantize_fp8 (step A1), which is timed on its own under "quantize".
 
 Default workload: batch 1, q_len 1, 64 heads, 128K context, FP8 E4M3 paged
-KV (page 64, shuffled block table), 64-way split.  The other four workloads
-are measured in the same run, each under its own key: "tiny" (batch 1, 16
-heads, 1024 tokens, bf16), "batch16" (batch 16 at 128K, FP8, 32-way split),
-"ragged_b32_bf16" (batch 32, 128 heads, ragged lengths, bf16) and
-"verify_q4_256k" (batch 8, q_len 4 causal, 256K, FP8; tensor-bound, so its
-roofline is against the bf16 tensor peak).  L2 is flushed (a 256 MiB write)
-before every timed step, outside the timed events, so the 75.5 MB batch-1
-cache is read from HBM.
+KV (page 64, shuffled block table).  The other four workloads are measured in
+the same run, each under its own key: "tiny" (batch 1, 16 heads, 1024 tokens,
+bf16), "batch16" (batch 16 at 128K, FP8), "ragged_b32_bf16" (batch 32, 128
+heads, ragged lengths, bf16) and "verify_q4_256k" (batch 8, q_len 4 causal,
+256K, FP8; tensor-bound, so its roofline is against the bf16 tensor peak).
+L2 is flushed (a 256 MiB write) before every timed step, outside the timed
+events, so the 75.5 MB batch-1 cache is read from HBM.
 
 value = KV bytes read per step (sum_b L_b * 576) over all ranks / step time,
 in GB/s; ms_per_step is the device time of one step (max over ranks).
@@ -230,13 +234,18 @@ def run_steps(w, kv, steps, warmup, flush_bytes=256 << 20):
 
 def run_single_launch(w, kv, steps, warmup, flush_bytes=256 << 20):
     """Per-step device times of the single-launch decode (mla_decode_fused),
-    L2 flushed before each step; None when the shape needs two kernels."""
+    L2 flushed before each step, and its split count; None when the shape has
+    no single launch (bf16 cache, or more row groups x requests than SMs)."""
     import torch
     import mla_split_kv_absorbed_b200 as m
     if w.spec.kv_dtype != "fp8":
         return None
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    S = m.mla_fused_splits(w.B, w.q_len, w.H, sms)
+    if S < 1:
+        return None
     stream = torch.cuda.current_stream()
-    ws_buf = m.alloc_fused_workspace(w.B, w.q_len, w.H, w.max_splits)
+    ws_buf = m.alloc_fused_workspace(w.B, w.q_len, w.H)
     out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
     out_lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
     flush = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
@@ -244,14 +253,7 @@ def run_single_launch(w, kv, steps, warmup, flush_bytes=256 << 20):
 
     def step():
         m.mla_decode_fused(w.q_nope, w.q_rope, kv, w.kv_scale, w.block_table, w.seq_lens,
-                           w.num_splits, w.max_splits, w.softmax_scale, ws_buf, out, out_lse, err,
-                           stream)
-    try:
-        step()
-    except m.MlaError as e:
-        if e.status == m.MLA_ERR_UNSUPPORTED:
-            return None
-        raise
+                           w.softmax_scale, ws_buf, out, out_lse, err, stream)
     for _ in range(warmup):
         flush.zero_()
         step()
@@ -266,20 +268,24 @@ def run_single_launch(w, kv, steps, warmup, flush_bytes=256 << 20):
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item())}")
-    return [a.elapsed_time(b) * 1e-3 for a, b in evs]
+    return [a.elapsed_time(b) * 1e-3 for a, b in evs], S
 
 
-def run_e2e(w, kv, steps, warmup):
+def run_e2e(w, kv, steps, warmup, fused):
     """Same step through the public API with host buffers: per step, pinned-host
-    -> device copies of the step's inputs (queries, seq_lens, num_splits,
-    block table), partial + combine, and device -> host copies of O and LSE.
-    The KV cache stays resident in HBM, as in serving."""
+    -> device copies of the step's inputs (queries, seq_lens, block table, and
+    num_splits for the two-kernel step), the decode call, and device -> host
+    copies of O and LSE.  The KV cache stays resident in HBM, as in serving."""
     import torch
     import mla_split_kv_absorbed_b200 as m
     stream = torch.cuda.current_stream()
-    h_in = [t.cpu().pin_memory() for t in (w.q_nope, w.q_rope, w.seq_lens, w.num_splits, w.block_table)]
+    src = [w.q_nope, w.q_rope, w.seq_lens, w.block_table] + ([] if fused else [w.num_splits])
+    h_in = [t.cpu().pin_memory() for t in src]
     d_in = [torch.empty_like(t, device="cuda") for t in h_in]
-    part = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
+    if fused:
+        fws = m.alloc_fused_workspace(w.B, w.q_len, w.H)
+    else:
+        part = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
     out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
     out_lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -291,8 +297,12 @@ def run_e2e(w, kv, steps, warmup):
     def step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        m.decode(d_in[0], d_in[1], kv, w.kv_scale, d_in[4], d_in[2], d_in[3], w.max_splits,
-                 w.softmax_scale, out=out, out_lse=out_lse, workspace=part)
+        if fused:
+            m.mla_decode_fused(d_in[0], d_in[1], kv, w.kv_scale, d_in[3], d_in[2],
+                               w.softmax_scale, fws, out, out_lse)
+        else:
+            m.decode(d_in[0], d_in[1], kv, w.kv_scale, d_in[3], d_in[2], d_in[4], w.max_splits,
+                     w.softmax_scale, out=out, out_lse=out_lse, workspace=part)
         h_out.copy_(out, non_blocking=True)
         h_lse.copy_(out_lse, non_blocking=True)
 
@@ -400,9 +410,35 @@ def flops_per_step(w):
     return 2 * (576 + 512) * tok_rows
 
 
+def roofline_of(w, name, t_kernel, peak_hbm, peak_tflops, kernel):
+    """Roofline of the dominant kernel over its launch time: KV bytes against
+    the HBM peak, or, for the q_len-4 verify, MMA flops against the tensor peak."""
+    if w.q_len > 1:
+        fl = flops_per_step(w)
+        return {"bound": "tensor", "achieved": fl / t_kernel / 1e12, "peak": peak_tflops,
+                "unit": "TFLOP/s", "frac": fl / t_kernel / 1e12 / peak_tflops,
+                "algorithmic_flops": fl, "kernel": kernel, "kernel_us": t_kernel * 1e6}
+    return {"bound": "hbm", "achieved": w.kv_bytes / t_kernel / 1e9, "peak": peak_hbm,
+            "unit": "GB/s", "frac": w.kv_bytes / t_kernel / 1e9 / peak_hbm,
+            "traffic": recorded_traffic(kernel, name), "algorithmic_bytes": w.kv_bytes,
+            "kernel": kernel, "kernel_us": t_kernel * 1e6}
+
+
+def two_kernel_summary(w, tot, par, ws, peak_hbm):
+    """The two-kernel step (partial + combine) with the workload's split count."""
+    t = max_over_ranks(statistics.median(tot), ws)
+    tp = max_over_ranks(statistics.median(par), ws)
+    return {"api": "mla_decode_partial + mla_combine", "num_splits": w.max_splits,
+            "us_per_step": t * 1e6, "us_p10": pct(tot, 0.1) * 1e6, "us_p90": pct(tot, 0.9) * 1e6,
+            "kv_gbs": w.kv_bytes / t / 1e9, "frac_of_peak": w.kv_bytes / t / 1e9 / peak_hbm,
+            "partial_us": tp * 1e6, "partial_p10": pct(par, 0.1) * 1e6,
+            "partial_p90": pct(par, 0.9) * 1e6, "partial_gbs": w.kv_bytes / tp / 1e9}
+
+
 def measure(name, steps, warmup, peak_hbm, peak_tflops, ws):
-    """One workload: step and partial-kernel times (median, p10, p90) and the
-    partial kernel's roofline (HBM, or tensor for the q_len-4 verify)."""
+    """One workload: the step through its own call (single launch where the
+    shape has one), the two-kernel step with the workload's split count, and
+    the dominant kernel's roofline."""
     import torch
     w, kv = setup_workload(name, "cuda")
     if w.spec.splits == "by_length":
@@ -410,25 +446,27 @@ def measure(name, steps, warmup, peak_hbm, peak_tflops, ws):
         import mla_split_kv_absorbed_b200 as m
         chosen = m.mla_choose_splits(w.seq_lens.cpu(), 148, 64)
         assert torch.equal(chosen, w.num_splits.cpu()), "mla_choose_splits disagrees with the workload"
+    single = run_single_launch(w, kv, steps, warmup)
     tot, par = run_steps(w, kv, steps, warmup)
-    t = max_over_ranks(statistics.median(tot), ws)
-    tp = max_over_ranks(statistics.median(par), ws)
-    res = {"workload": name, "B": w.B, "q_len": w.q_len, "H": w.H, "kv": w.spec.kv_dtype,
-           "num_splits": w.max_splits, "kv_bytes_per_step": w.kv_bytes, "steps": steps,
-           "us_per_step": t * 1e6, "us_p10": pct(tot, 0.1) * 1e6, "us_p90": pct(tot, 0.9) * 1e6,
-           "kv_gbs": w.kv_bytes / t / 1e9, "frac_of_peak": w.kv_bytes / t / 1e9 / peak_hbm,
-           "partial_us": tp * 1e6, "partial_p10": pct(par, 0.1) * 1e6,
-           "partial_p90": pct(par, 0.9) * 1e6, "partial_gbs": w.kv_bytes / tp / 1e9}
+    two = two_kernel_summary(w, tot, par, ws, peak_hbm)
     kernel = "decode_fp8_kernel" if w.spec.kv_dtype == "fp8" else "decode_bf16_kernel"
-    if w.q_len > 1:
-        fl = flops_per_step(w)
-        res["roofline"] = {"bound": "tensor", "achieved": fl / tp / 1e12, "peak": peak_tflops,
-                           "unit": "TFLOP/s", "frac": fl / tp / 1e12 / peak_tflops,
-                           "algorithmic_flops": fl, "kernel": kernel}
+    res = {"workload": name, "B": w.B, "q_len": w.q_len, "H": w.H, "kv": w.spec.kv_dtype,
+           "kv_bytes_per_step": w.kv_bytes, "steps": steps}
+    if single is not None:
+        times, S = single
+        t = max_over_ranks(statistics.median(times), ws)
+        res.update({"api": "mla_decode_fused", "num_splits": S, "us_per_step": t * 1e6,
+                    "us_p10": pct(times, 0.1) * 1e6, "us_p90": pct(times, 0.9) * 1e6})
+        res["roofline"] = roofline_of(w, name, t, peak_hbm, peak_tflops, kernel)
     else:
-        res["roofline"] = {"bound": "hbm", "achieved": w.kv_bytes / tp / 1e9, "peak": peak_hbm,
-                           "unit": "GB/s", "frac": w.kv_bytes / tp / 1e9 / peak_hbm,
-                           "traffic": recorded_traffic(kernel, name), "kernel": kernel}
+        t = two["us_per_step"] * 1e-6
+        res.update({"api": two["api"], "num_splits": w.max_splits, "us_per_step": two["us_per_step"],
+                    "us_p10": two["us_p10"], "us_p90": two["us_p90"]})
+        res["roofline"] = roofline_of(w, name, two["partial_us"] * 1e-6, peak_hbm, peak_tflops,
+                                      kernel)
+    res["kv_gbs"] = w.kv_bytes / t / 1e9
+    res["frac_of_peak"] = w.kv_bytes / t / 1e9 / peak_hbm
+    res["two_kernel"] = two
     del kv, w
     torch.cuda.empty_cache()
     return res
@@ -506,22 +544,37 @@ def main():
 
     w, kv = setup_workload(args.workload, "cuda")
     quant = time_quantize(w, kv) if w.spec.kv_dtype == "fp8" else None
+    import mla_split_kv_absorbed_b200 as m
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    fused = w.spec.kv_dtype == "fp8" and m.mla_fused_splits(w.B, w.q_len, w.H, sms) >= 1
 
+    # the timed region: K steps through the workload's own call
     barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         t0 = time.perf_counter()
-        total, partial = run_steps(w, kv, args.steps, args.warmup)
+        if fused:
+            times, S = run_single_launch(w, kv, args.steps, args.warmup)
+            t_kernel_list = times
+        else:
+            times, t_kernel_list = run_steps(w, kv, args.steps, args.warmup)
+            S = w.max_splits
         wall = time.perf_counter() - t0
     torch.cuda.synchronize()
     barrier(ws)
-    t_step = max_over_ranks(statistics.median(total), ws)
-    t_partial = max_over_ranks(statistics.median(partial), ws)
+    t_step = max_over_ranks(statistics.median(times), ws)
+    t_kernel = max_over_ranks(statistics.median(t_kernel_list), ws)
     value = job_gbs(w.kv_bytes, t_step, ws)
 
-    e2e_t, h2d, d2h = run_e2e(w, kv, max(5, args.steps // 2), args.warmup)
+    # the two-kernel step with the workload's own split count, for context
+    if fused:
+        tot, par = run_steps(w, kv, args.steps, args.warmup)
+    else:
+        tot, par = times, t_kernel_list
+    two = two_kernel_summary(w, tot, par, ws, peak)
+
+    e2e_t, h2d, d2h = run_e2e(w, kv, max(5, args.steps // 2), args.warmup, fused)
     e2e_t = max_over_ranks(e2e_t, ws)
-    single = run_single_launch(w, kv, args.steps, args.warmup)
 
     extra = {}
     if not args.no_extra:
@@ -535,8 +588,12 @@ def main():
     if rank == 0 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, host_codes(w, kv))
 
-    achieved = w.kv_bytes / t_partial / 1e9
     kernel_name = "decode_fp8_kernel" if w.spec.kv_dtype == "fp8" else "decode_bf16_kernel"
+    roof = roofline_of(w, args.workload, t_kernel, peak, peak_tf, kernel_name)
+    roof.update({"kernel_p10": pct(t_kernel_list, 0.1) * 1e6,
+                 "kernel_p90": pct(t_kernel_list, 0.9) * 1e6, "peak_kind": peak_kind,
+                 "launch": "the whole step (single launch)" if fused else
+                           "the partial kernel of the two-kernel step"})
     line = {
         "metric": METRIC,
         "value": value,
@@ -546,8 +603,8 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": t_step * 1e3,
         "us_per_step": t_step * 1e6,
-        "us_p10": pct(total, 0.1) * 1e6,
-        "us_p90": pct(total, 0.9) * 1e6,
+        "us_p10": pct(times, 0.1) * 1e6,
+        "us_p90": pct(times, 0.9) * 1e6,
         "frac_of_peak": w.kv_bytes / t_step / 1e9 / peak,
         "higher_is_better": True,
         "scaling": "weak",
@@ -555,29 +612,20 @@ def main():
         "dtype": "e4m3" if w.spec.kv_dtype == "fp8" else "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "B": w.B, "q_len": w.q_len, "H": w.H,
-                   "seq_len": int(w.seq_lens.max().item()), "num_splits": w.max_splits,
-                   "kv": w.spec.kv_dtype, "page": 64, "kv_bytes_per_step": w.kv_bytes,
+                   "seq_len": int(w.seq_lens.max().item()), "kv": w.spec.kv_dtype, "page": 64,
+                   "kv_bytes_per_step": w.kv_bytes,
+                   "api": "mla_decode_fused" if fused else "mla_decode_partial + mla_combine",
+                   "num_splits": S, "workload_num_splits": w.max_splits,
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
                    "parallelism": f"replicas x{ws}"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak,
-                     "traffic": recorded_traffic(kernel_name, args.workload),
-                     "algorithmic_bytes": w.kv_bytes,
-                     "kernel": kernel_name, "kernel_us": t_partial * 1e6,
-                     "kernel_p10": pct(partial, 0.1) * 1e6, "kernel_p90": pct(partial, 0.9) * 1e6,
-                     "peak_kind": peak_kind},
+        "roofline": roof,
         "e2e": {"value": ws * w.kv_bytes / e2e_t / 1e9, "unit": "GB/s", "us_per_step": e2e_t * 1e6,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 if fused else 2) * args.steps,
         "clocks": clk.summary(),
         "timed_wall_s": wall,
+        "two_kernel": two,
     }
-    if single is not None:
-        ts = max_over_ranks(statistics.median(single), ws)
-        line["single_launch"] = {
-            "api": "mla_decode_fused", "us_per_step": ts * 1e6,
-            "us_p10": pct(single, 0.1) * 1e6, "us_p90": pct(single, 0.9) * 1e6,
-            "kv_gbs": job_gbs(w.kv_bytes, ts, ws), "frac_of_peak": w.kv_bytes / ts / 1e9 / peak}
     if quant is not None:
         line["quantize"] = quant
     line.update(extra)
@@ -623,7 +671,9 @@ def reference_arm(args):
         "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "B": w.B, "q_len": w.q_len, "H": w.H,
-                   "seq_len": int(sl.max()), "num_splits": w.max_splits, "kv": w.spec.kv_dtype},
+                   "seq_len": int(sl.max()), "kv": w.spec.kv_dtype, "page": 64,
+                   "kv_bytes_per_step": w.kv_bytes, "api": "oracle (fp64, unsplit)",
+                   "workload_num_splits": w.max_splits},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

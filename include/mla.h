@@ -162,32 +162,40 @@ MLA_API int mla_combine(const float* part_o, const float* part_lse, const int32_
 /* ---------------------------------------------------------------------------
  * Single-launch decode, steps A2-A9 in one kernel ("SGLang & Miles ... Vera
  * Rubin" article, section "Vera Rubin 的三处硬件变化": kernel launches are
- * among the overheads the team removed).  Arguments and outputs are those of
- * mla_decode_partial followed by mla_combine.  The grid must fit on the GPU
- * at once: an FP8 cache (kv_dtype 0) and few enough (64-row query group,
- * split, request) units that each is cut across 2 or 4 CTAs (at most half as
- * many units as SMs, e.g. batch 1 with 64 heads and 64 splits on 148 SMs) and
- * max_splits * pieces <= 256.  Otherwise it returns MLA_ERR_UNSUPPORTED and
- * launches nothing: use mla_decode_partial + mla_combine.
- * The kernel is a cooperative launch.  Every CTA writes its own partial
- * (O/l and LSE of its run of tiles) to the workspace, the CTAs meet at a
- * grid barrier (a counter in the workspace, bounded wait), and the grid then
- * merges each row's partials as mla_combine does, in a fixed order
- * (deterministic); the result equals partial + combine up to rounding.
- *   workspace: mla_fused_workspace_bytes(B, q_len, H, max_splits) bytes,
- *     16-byte aligned; its first 8 bytes (two int32 counters) must be zero
- *     before the first call; every call that completes leaves them zero.
- *     After MLA_DEVERR_TIMEOUT, zero them again before the next call.  Calls
- *     that share a workspace must not overlap on the GPU.
+ * among the overheads the team removed).  The call picks its own partition:
+ * every request is cut into S equal page ranges (step A2 with the same S for
+ * all requests), S = min(256, floor(SMs / (G * B))), G = ceil(q_len*H / 64)
+ * query-row groups, SMs those of the current device, so that the grid holds
+ * one CTA per (row group, split, request) and is a single wave: every CTA is
+ * resident at once and none waits for a free SM.  Requires an FP8 cache
+ * (kv_dtype 0) and S >= 1 (G * B <= SMs, e.g. batch 16 with 64 heads and
+ * one query token per request on 148 SMs gives S = 9); otherwise it returns
+ * MLA_ERR_UNSUPPORTED and launches nothing: use mla_decode_partial +
+ * mla_combine.  Other arguments and the outputs are those of
+ * mla_decode_partial followed by mla_combine.
+ * The kernel is a cooperative launch.  Every CTA writes the partial of its
+ * split (O/l and LSE) to the workspace, the CTAs meet at a grid barrier (a
+ * counter in the workspace, bounded wait), and the grid then merges each
+ * row's S partials as mla_combine does, in a fixed order (deterministic); the
+ * result equals partial + combine with S splits up to rounding.
+ *   mla_fused_splits: the S that a call with these sizes uses on a GPU with
+ *     num_sms SMs (0: no single launch for these sizes).
+ *   workspace: mla_fused_workspace_bytes(B, q_len, H, num_sms) bytes with the
+ *     current device's SM count (256 + B*q_len*H*S*513*4; 0 when S = 0),
+ *     passed with its size; 16-byte aligned; its first 8 bytes (two int32
+ *     counters) must be zero before the first call; every call that
+ *     completes leaves them zero.  After MLA_DEVERR_TIMEOUT, zero them again
+ *     before the next call.  Calls that share a workspace must not overlap on
+ *     the GPU.  A workspace smaller than the call needs: MLA_ERR_INVALID_ARG.
  *   out_bf16 [B][q_len][H][512], out_lse [B][q_len][H] (nullable).
  * ------------------------------------------------------------------------- */
-MLA_API size_t mla_fused_workspace_bytes(int B, int q_len, int H, int max_splits);
+MLA_API int mla_fused_splits(int B, int q_len, int H, int num_sms);
+MLA_API size_t mla_fused_workspace_bytes(int B, int q_len, int H, int num_sms);
 MLA_API int mla_decode_fused(const uint16_t* q_nope, const uint16_t* q_rope,
                              const void* kv_pages, int kv_dtype, float kv_scale,
                              int64_t num_pages, const int32_t* block_table,
-                             int max_pages_per_req, const int32_t* seq_lens,
-                             const int32_t* num_splits, int max_splits, int B, int q_len,
-                             int H, float softmax_scale, void* workspace,
+                             int max_pages_per_req, const int32_t* seq_lens, int B, int q_len,
+                             int H, float softmax_scale, void* workspace, size_t workspace_bytes,
                              uint16_t* out_bf16, float* out_lse, int32_t* dev_error,
                              void* stream);
 

@@ -318,7 +318,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
   const int b = unit / (args.groups * args.max_splits);
   // ---------------------------------------------------------------- split range (step A2)
   const int L = args.seq_lens[b];
-  const int S_b = args.num_splits[b];
+  const int S_b = args.splits_const > 0 ? args.splits_const : args.num_splits[b];
   if (S_b < 1 || S_b > args.max_splits) {
     if (tid == 0 && s == 0 && g == 0 && piece == 0) set_error(args.dev_error, MLA_DEVERR_BAD_SPLITS);
     return;
@@ -1020,7 +1020,7 @@ __device__ __forceinline__ void fused_merge(const DecodeArgs& a, uint8_t* smem) 
          item += kMergeGroups * (int)gridDim.x) {
       const int row = item >> 2, d = (item & 3) * 128 + t;
       const int bq = row / QH;
-      int S = a.num_splits[bq];
+      int S = a.splits_const > 0 ? a.splits_const : a.num_splits[bq];
       S = S < 1 ? 0 : (S > a.max_splits ? a.max_splits : S);
       const int E = S * a.pieces;  // entries of this row, at most 256
       const float* po = a.part_o + (int64_t)row * slots * 512 + d;

@@ -61,6 +61,7 @@ struct DecodeArgs {
   // sync[0] the grid merges them into out / out_lse; sync[1] counts the CTAs
   // that have finished, and the last one resets both to zero.
   int fused;
+  int splits_const;     // > 0: every request has this many splits (num_splits is not read)
   uint16_t* out;        // [rows][512] bf16
   float* out_lse;       // [rows], may be null
   int32_t* sync;        // two counters, zero before the launch

@@ -142,9 +142,11 @@ int setup_decode(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_
                  float kv_scale, int64_t num_pages, const int32_t* block_table,
                  int max_pages_per_req, const int32_t* seq_lens, const int32_t* num_splits,
                  int max_splits, int B, int q_len, int H, float softmax_scale,
-                 int32_t* dev_error, mla::DecodeArgs* a, CUtensorMap* map, CUtensorMap* rope_map) {
+                 int32_t* dev_error, mla::DecodeArgs* a, CUtensorMap* map, CUtensorMap* rope_map,
+                 int splits_const = 0) {
+  // splits_const > 0: every request has max_splits splits and num_splits is unused
   if (q_nope == nullptr || q_rope == nullptr || kv_pages == nullptr || block_table == nullptr ||
-      seq_lens == nullptr || num_splits == nullptr)
+      seq_lens == nullptr || (num_splits == nullptr && splits_const == 0))
     return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(kv_pages)) return MLA_ERR_INVALID_ARG;
   if (B <= 0 || q_len <= 0 || H <= 0 || num_pages <= 0 || max_pages_per_req <= 0 ||
@@ -179,6 +181,7 @@ int setup_decode(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_
   a->block_table = block_table;
   a->seq_lens = seq_lens;
   a->num_splits = num_splits;
+  a->splits_const = splits_const > 0 ? max_splits : 0;
   a->dev_error = dev_error;
   a->num_pages = num_pages;
   a->max_pages = max_pages_per_req;
@@ -199,7 +202,7 @@ int setup_decode(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_
 }
 
 constexpr size_t kFusedCounterBytes = 256;  // two int32 counters, padded
-constexpr int kFusedMaxPieces = 4;
+constexpr int kFusedMaxEntries = 256;       // splits per row the single launch's merge takes
 
 }  // namespace
 
@@ -249,31 +252,63 @@ int mla_decode_partial_q8(const uint8_t* q8, float q_scale, const void* kv_pages
   return status_of(mla::launch_decode_fp8(a, map, rope_map, static_cast<cudaStream_t>(stream)));
 }
 
-size_t mla_fused_workspace_bytes(int B, int q_len, int H, int max_splits) {
-  if (B <= 0 || q_len <= 0 || H <= 0 || max_splits <= 0) return 0;
-  const size_t entries = (size_t)B * q_len * H * max_splits * kFusedMaxPieces;
+}  // extern "C"
+
+namespace {
+
+// Split count of the single launch: every request cut into as many splits as
+// one wave of CTAs allows, one CTA per (row group, split, request).
+int fused_splits(int B, int q_len, int H, int num_sms) {
+  const long long units_per_split = (long long)((q_len * H + 63) / 64) * B;
+  if (units_per_split <= 0 || num_sms <= 0) return 0;
+  long long S = num_sms / units_per_split;
+  return (int)(S > kFusedMaxEntries ? kFusedMaxEntries : S);
+}
+
+size_t fused_bytes(int B, int q_len, int H, int S) {
+  const size_t entries = (size_t)B * q_len * H * S;
   return kFusedCounterBytes + entries * 512 * sizeof(float) + entries * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_fused_splits(int B, int q_len, int H, int num_sms) {
+  if (B <= 0 || q_len <= 0 || H <= 0 || num_sms <= 0) return 0;
+  return fused_splits(B, q_len, H, num_sms);
+}
+
+size_t mla_fused_workspace_bytes(int B, int q_len, int H, int num_sms) {
+  if (B <= 0 || q_len <= 0 || H <= 0 || num_sms <= 0) return 0;
+  const int S = fused_splits(B, q_len, H, num_sms);
+  return S < 1 ? 0 : fused_bytes(B, q_len, H, S);
 }
 
 int mla_decode_fused(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_pages,
                      int kv_dtype, float kv_scale, int64_t num_pages, const int32_t* block_table,
-                     int max_pages_per_req, const int32_t* seq_lens, const int32_t* num_splits,
-                     int max_splits, int B, int q_len, int H, float softmax_scale, void* workspace,
+                     int max_pages_per_req, const int32_t* seq_lens, int B, int q_len, int H,
+                     float softmax_scale, void* workspace, size_t workspace_bytes,
                      uint16_t* out_bf16, float* out_lse, int32_t* dev_error, void* stream) {
   if (workspace == nullptr || out_bf16 == nullptr || !aligned16(workspace))
     return MLA_ERR_INVALID_ARG;
+  if (B <= 0 || q_len <= 0 || H <= 0) return MLA_ERR_INVALID_ARG;
+  // one launch only when every CTA of the grid is resident at once: an FP8
+  // cache and at least one split per (row group, request) in one wave
+  const int S = fused_splits(B, q_len, H, num_sms_current_device());
+  if (kv_dtype != MLA_KV_FP8_E4M3 || S < 1) return MLA_ERR_UNSUPPORTED;
+  if (workspace_bytes < fused_bytes(B, q_len, H, S)) return MLA_ERR_INVALID_ARG;
   mla::DecodeArgs a;
   CUtensorMap map, rope_map;
   const int st = setup_decode(q_nope, q_rope, kv_pages, kv_dtype, kv_scale, num_pages, block_table,
-                              max_pages_per_req, seq_lens, num_splits, max_splits, B, q_len, H,
-                              softmax_scale, dev_error, &a, &map, &rope_map);
+                              max_pages_per_req, seq_lens, nullptr, S, B, q_len, H,
+                              softmax_scale, dev_error, &a, &map, &rope_map, /*splits_const=*/1);
   if (st != MLA_OK) return st;
-  // one launch only when every CTA of the grid is resident at once: an FP8
-  // cache and a grid that fits in one wave (every unit cut into pieces)
-  if (kv_dtype != MLA_KV_FP8_E4M3 || a.split_from != 0 || a.pieces < 2 ||
-      max_splits * a.pieces > 256)
-    return MLA_ERR_UNSUPPORTED;
-  const size_t entries = (size_t)B * q_len * H * max_splits * kFusedMaxPieces;
+  const int units = a.groups * S * B;
+  a.pieces = 1;  // one CTA per unit, no cluster: the grid is exactly one wave
+  a.split_from = units;
+  a.pad = 0;
+  const size_t entries = (size_t)B * q_len * H * S;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.fused = 1;
   a.sync = reinterpret_cast<int32_t*>(ws);

@@ -122,19 +122,37 @@ def test_rejections_without_gpu(lib):
 def test_fused_workspace_and_rejections_without_gpu(lib):
     h = lib.load()
     null = None
-    # counters (256 bytes) + room for 4 pieces per split: O (512 fp32) and LSE per entry
-    assert h.mla_fused_workspace_bytes(1, 1, 64, 64) == 256 + 64 * 64 * 4 * 513 * 4
-    assert h.mla_fused_workspace_bytes(2, 4, 16, 8) == 256 + 2 * 4 * 16 * 8 * 4 * 513 * 4
-    assert h.mla_fused_workspace_bytes(0, 1, 64, 64) == 0
+    # one wave of one CTA per (64-row group, split, request), at most 256 splits
+    assert h.mla_fused_splits(1, 1, 64, 148) == 148
+    assert h.mla_fused_splits(16, 1, 64, 148) == 9
+    assert h.mla_fused_splits(2, 4, 64, 148) == 18     # 4 row groups per request
+    assert h.mla_fused_splits(148, 1, 64, 148) == 1
+    assert h.mla_fused_splits(149, 1, 64, 148) == 0
+    assert h.mla_fused_splits(1, 1, 16, 1000) == 256
+    assert h.mla_fused_splits(0, 1, 64, 148) == 0
+    assert h.mla_fused_splits(1, 1, 64, 0) == 0
+    # counters (256 bytes) + O (512 fp32) and LSE per (row, split)
+    assert h.mla_fused_workspace_bytes(1, 1, 64, 148) == 256 + 64 * 148 * 513 * 4
+    assert h.mla_fused_workspace_bytes(16, 1, 64, 148) == 256 + 16 * 64 * 9 * 513 * 4
+    assert h.mla_fused_workspace_bytes(2, 4, 16, 148) == 256 + 2 * 4 * 16 * 74 * 513 * 4  # one row group
+    assert h.mla_fused_workspace_bytes(149, 1, 64, 148) == 0
+    assert h.mla_fused_workspace_bytes(0, 1, 64, 148) == 0
     fake = ctypes.c_void_p(1 << 20)
-    base = [fake, fake, fake, 0, 1.0, 10, fake, 4, fake, fake, 4, 1]
+    big = 1 << 40
+    base = [fake, fake, fake, 0, 1.0, 10, fake, 4, fake, 1]
     # null workspace / output, misaligned workspace
-    assert h.mla_decode_fused(*base, 1, 64, 1.0, null, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
-    assert h.mla_decode_fused(*base, 1, 64, 1.0, fake, null, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, null, big, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, fake, big, null, null, null, null) == lib.MLA_ERR_INVALID_ARG
     mis = ctypes.c_void_p((1 << 20) + 8)
-    assert h.mla_decode_fused(*base, 1, 64, 1.0, mis, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, mis, big, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
+    # a bf16 cache has no single launch
+    b16 = [fake, fake, fake, 1, 1.0, 10, fake, 4, fake, 1]
+    assert h.mla_decode_fused(*b16, 1, 64, 1.0, fake, big, fake, null, null, null) == lib.MLA_ERR_UNSUPPORTED
+    # a workspace one byte short (the SM count without a GPU is taken as 148)
+    need = h.mla_fused_workspace_bytes(1, 1, 64, 148)
+    assert h.mla_decode_fused(*base, 1, 64, 1.0, fake, need - 1, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
     # the shared checks of mla_decode_partial apply
-    assert h.mla_decode_fused(*base, 5, 64, 1.0, fake, fake, null, null, null) == lib.MLA_ERR_UNSUPPORTED
+    assert h.mla_decode_fused(*base, 5, 64, 1.0, fake, big, fake, null, null, null) == lib.MLA_ERR_UNSUPPORTED
 
 
 def test_q8_rejections_without_gpu(lib):

@@ -67,15 +67,15 @@ def test_single_launch_with_a_stalled_piece_reports_and_resets_its_counters():
     import mla_split_kv_absorbed_b200 as m
     c = make_case("b1_128k_fp8", seq_lens=[8192], splits=4)
     w = c.w
-    ws = m.alloc_fused_workspace(w.B, w.q_len, w.H, w.max_splits)
+    ws = m.alloc_fused_workspace(w.B, w.q_len, w.H)
     out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def fused():
         m.mla_decode_fused(c.dev["q_nope"], c.dev["q_rope"], c.kv_dev, w.kv_scale,
-                           c.dev["block_table"], c.dev["seq_lens"], c.dev["num_splits"],
-                           w.max_splits, w.softmax_scale, ws, out, lse, err)
+                           c.dev["block_table"], c.dev["seq_lens"], w.softmax_scale, ws, out,
+                           lse, err)
 
     torch.cuda.synchronize()
     prev = m.mla_debug_inject_stall(True)

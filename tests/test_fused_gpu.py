@@ -1,42 +1,60 @@
 """Single-launch decode (mla_decode_fused) on the GPU against the oracle.
 
-The fused path runs steps A2-A9 in one cooperative launch: every piece of
-every unit writes its own partial, the grid meets at a barrier, and the grid
-merges the partials.  It applies when the grid fits on the GPU at once (every
-unit cut into 2 or 4 pieces), as at batch 1; other shapes are refused with
+The fused path runs steps A2-A9 in one cooperative launch.  It cuts every
+request into S = floor(SMs / (row groups x B)) equal page ranges (at most 256),
+so the grid is one wave of one CTA per (row group, split, request): every CTA
+writes its split's partial, the grid meets at a barrier and merges them.
+Shapes with more (row group, request) pairs than SMs are refused with
 MLA_ERR_UNSUPPORTED.
 """
 import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import assert_attention_close, make_case, oracle_rows, run_gpu
+from gpu_helpers import assert_attention_close, make_case, oracle_rows
 
 pytestmark = pytest.mark.gpu
 
 SMALL = [
-    ("b1_128k_fp8", dict(seq_lens=[2085], splits=4)),             # 4 units, 4 pieces each
-    ("b1_128k_fp8", dict(seq_lens=[700], splits=3)),              # pieces of one tile and empty ones
-    ("b1_128k_fp8", dict(seq_lens=[100], splits=8)),              # more splits than pages
-    ("b16_128k_fp8", dict(seq_lens=[5000, 130, 1, 777], splits=4)),
-    ("verify_q4_256k_fp8", dict(seq_lens=[777], splits=3, H=16)),  # q_len 4, causal
-    ("verify_q4_256k_fp8", dict(seq_lens=[1000, 4], splits=2)),  # four row groups
+    ("b1_128k_fp8", dict(seq_lens=[2085])),                 # 148 splits over 33 pages: most empty
+    ("b1_128k_fp8", dict(seq_lens=[100])),                  # one page with a ragged tail
+    ("b1_128k_fp8", dict(seq_lens=[64 * 148 * 2 + 5])),     # 2 pages per split, ragged last split
+    ("b16_128k_fp8", dict(seq_lens=[5000, 130, 1, 777])),    # 37 splits each
+    ("verify_q4_256k_fp8", dict(seq_lens=[777], H=16)),     # q_len 4, causal, one row group
+    ("verify_q4_256k_fp8", dict(seq_lens=[1000, 4])),       # four row groups, 18 splits
+    ("b16_128k_fp8", dict(seq_lens=[300] * 148)),           # one split per request
 ]
+
+
+def sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
 
 
 def run_fused(c, workspace=None):
     import mla_split_kv_absorbed_b200 as m
     w = c.w
     if workspace is None:
-        workspace = m.alloc_fused_workspace(w.B, w.q_len, w.H, w.max_splits)
+        workspace = m.alloc_fused_workspace(w.B, w.q_len, w.H)
     out = torch.full((w.B, w.q_len, w.H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((w.B, w.q_len, w.H), float("nan"), dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     m.mla_decode_fused(c.dev["q_nope"], c.dev["q_rope"], c.kv_dev, w.kv_scale, c.dev["block_table"],
-                       c.dev["seq_lens"], c.dev["num_splits"], w.max_splits, w.softmax_scale,
-                       workspace, out, lse, err)
+                       c.dev["seq_lens"], w.softmax_scale, workspace, out, lse, err)
     torch.cuda.synchronize()
     return out, lse, int(err.item()), workspace
+
+
+def run_two_launch(c, S):
+    """partial + combine with the fused call's split count S for every request."""
+    import mla_split_kv_absorbed_b200 as m
+    w = c.w
+    ns = torch.full((w.B,), S, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = m.decode(c.dev["q_nope"], c.dev["q_rope"], c.kv_dev, w.kv_scale,
+                        c.dev["block_table"], c.dev["seq_lens"], ns, S, w.softmax_scale,
+                        dev_error=err)
+    torch.cuda.synchronize()
+    return out, lse, int(err.item())
 
 
 def _ids(c):
@@ -46,17 +64,20 @@ def _ids(c):
 
 @pytest.mark.parametrize("case", SMALL, ids=[_ids(c) for c in SMALL])
 def test_fused_small_matches_oracle_and_two_launch_path(case):
+    import mla_split_kv_absorbed_b200 as m
     spec, ov = case
     c = make_case(spec, **ov)
     w = c.w
+    S = m.mla_fused_splits(w.B, w.q_len, w.H, sms())
+    assert S >= 1
     out, lse, err, ws = run_fused(c)
     assert err == 0
     rows = np.arange(w.B * w.q_len * w.H)
     o_ref, l_ref = oracle_rows(c, rows)
     assert_attention_close(out.float().cpu().numpy().reshape(-1, 512), lse.cpu().numpy().reshape(-1),
                            o_ref, l_ref, what=str(case))
-    # the same result as partial + combine, up to the order of the merge
-    out2, lse2, _, _, err2 = run_gpu(c)
+    # the same result as partial + combine with S splits, up to the order of the merge
+    out2, lse2, err2 = run_two_launch(c, S)
     assert err2 == 0
     d = (out.float() - out2.float()).abs()
     assert float(d.max()) <= 2.0 ** -6 * max(1.0, float(out2.float().abs().max()))
@@ -69,7 +90,7 @@ def test_fused_small_matches_oracle_and_two_launch_path(case):
 
 
 def test_fused_is_bitwise_deterministic_and_reuses_its_workspace():
-    c = make_case("b16_128k_fp8", seq_lens=[5000, 3000], splits=3)
+    c = make_case("b16_128k_fp8", seq_lens=[5000, 3000])
     a = run_fused(c)
     b = run_fused(c, workspace=a[3])
     assert a[2] == 0 and b[2] == 0
@@ -77,18 +98,31 @@ def test_fused_is_bitwise_deterministic_and_reuses_its_workspace():
     assert torch.equal(a[1], b[1])
 
 
-def test_fused_refuses_grids_that_do_not_fit():
+def test_fused_refuses_shapes_without_a_single_wave_and_small_workspaces():
     import mla_split_kv_absorbed_b200 as m
-    # batch 16 x 32 splits = 512 units: more than one wave
-    c = make_case("b16_128k_fp8", seq_lens=[300] * 16, splits=32)
+    n = sms()
+    # one more request than SMs: not even one split per request fits in a wave
+    c = make_case("b16_128k_fp8", seq_lens=[70] * (n + 1))
+    assert m.mla_fused_splits(c.w.B, 1, c.w.H, n) == 0
     with pytest.raises(m.MlaError) as e:
-        run_fused(c)
+        run_fused(c, workspace=torch.zeros(4096, dtype=torch.uint8, device="cuda"))
     assert e.value.status == m.MLA_ERR_UNSUPPORTED
+    with pytest.raises(m.MlaError) as e:
+        m.alloc_fused_workspace(c.w.B, 1, c.w.H)
+    assert e.value.status == m.MLA_ERR_UNSUPPORTED
+    # a workspace one byte short of what the call needs
+    c = make_case("b16_128k_fp8", seq_lens=[300, 200])
+    need = m.mla_fused_workspace_bytes(2, 1, c.w.H, n)
+    with pytest.raises(m.MlaError) as e:
+        run_fused(c, workspace=torch.zeros(need - 1, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == m.MLA_ERR_INVALID_ARG
 
 
-def test_fused_full_size_batch1_sampled_rows():
-    # the batch-1 benchmark workload (64 splits, 2 pieces each: 128 CTAs)
-    c = make_case("b1_128k_fp8", gen_device="cuda")
+@pytest.mark.parametrize("spec", ["b1_128k_fp8", "b16_128k_fp8"])
+def test_fused_full_size_sampled_rows(spec):
+    # the benchmark workloads at full size, in the launch the benchmark times
+    # (batch 1: 148 splits; batch 16: 9 splits, 144 CTAs on 148 SMs)
+    c = make_case(spec, gen_device="cuda")
     w = c.w
     out, lse, err, ws = run_fused(c)
     assert err == 0
@@ -98,5 +132,5 @@ def test_fused_full_size_batch1_sampled_rows():
     o_ref, l_ref = oracle_rows(c, rows)
     o = out.float().cpu().numpy().reshape(R, 512)[rows]
     l = lse.cpu().numpy().reshape(R)[rows]
-    assert_attention_close(o, l, o_ref, l_ref, what="b1 fused")
+    assert_attention_close(o, l, o_ref, l_ref, what=spec + " fused")
     assert torch.count_nonzero(ws[:8]).item() == 0
