@@ -174,14 +174,16 @@ MLA_API int mla_combine(const float* part_o, const float* part_lse, const int32_
  * mla_combine.  Other arguments and the outputs are those of
  * mla_decode_partial followed by mla_combine.
  * The kernel is a cooperative launch.  Every CTA writes the partial of its
- * split (O/l and LSE) to the workspace, the CTAs meet at a grid barrier (a
+ * split (O/l, as fp16 in units of kv_scale, and the fp32 LSE) to the workspace, the CTAs meet at a grid barrier (a
  * counter in the workspace, bounded wait), and the grid then merges each
  * row's S partials as mla_combine does, in a fixed order (deterministic); the
  * result equals partial + combine with S splits up to rounding.
  *   mla_fused_splits: the S that a call with these sizes uses on a GPU with
  *     num_sms SMs (0: no single launch for these sizes).
  *   workspace: mla_fused_workspace_bytes(B, q_len, H, num_sms) bytes with the
- *     current device's SM count (256 + B*q_len*H*S*513*4; 0 when S = 0),
+ *     current device's SM count (256 + B*q_len*H*S*(512*2 + 4): per (row,
+ *     split) the partial O as fp16 in units of kv_scale and its fp32 LSE; 0
+ *     when S = 0),
  *     passed with its size; 16-byte aligned; its first 8 bytes (two int32
  *     counters) must be zero before the first call; every call that
  *     completes leaves them zero.  After MLA_DEVERR_TIMEOUT, zero them again
@@ -335,6 +337,16 @@ MLA_API int mla_partial_grid(int B, int q_len, int H, int max_splits, int kv_dty
  * Returns the previous setting.  Process-wide; not for production use.
  * ------------------------------------------------------------------------- */
 MLA_API int mla_debug_inject_stall(int enable);
+
+/* mla_debug_merge_plan: a test hook with no counterpart on the pages.  The
+ * merge inside mla_decode_fused runs each row's entries as items of 128*v
+ * dims (v = 1, 2 or 4 dims per thread), gpi = 1, 2, 3 or 6 128-thread groups
+ * per item, and picks (v, gpi) per launch from the shape.  While set, every
+ * later mla_decode_fused call uses the given plan instead, so that tests can
+ * run each one; (0, 0) restores the automatic choice.  Every plan gives the
+ * same result up to the order of the sums.  Returns MLA_ERR_INVALID_ARG for
+ * other values.  Process-wide; not for production use. */
+MLA_API int mla_debug_merge_plan(int v, int gpi);
 
 /* Static, human-readable name of a status code. */
 MLA_API const char* mla_status_string(int status);

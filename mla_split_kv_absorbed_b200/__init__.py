@@ -25,6 +25,7 @@ Entry points (same names as the C ABI):
   the GPU's error word into MLA_ERR_DEVICE.
 * ``mla_partial_grid(...)`` — host helper: the partial kernel's CTA layout for a shape.
 * ``mla_debug_inject_stall(enable)`` — test hook for the bounded-wait failure path.
+* ``mla_debug_merge_plan(v, gpi)`` — test hook: force the single launch's merge plan.
 
 ``mla_decode_noalloc`` (partial + merge with in-library scratch) is reached
 through ``load()`` directly; its ctypes signature is in the GPU test that uses
@@ -50,7 +51,7 @@ DEVERR_BAD_PAGE, DEVERR_BAD_SEQLEN, DEVERR_TIMEOUT, DEVERR_BAD_SPLITS, DEVERR_SM
 
 EXPORTS = ("mla_quantize_fp8", "mla_partial_workspace_bytes", "mla_decode_partial",
            "mla_combine", "mla_choose_splits", "mla_device_error_status", "mla_status_string",
-           "mla_decode_noalloc", "mla_partial_grid", "mla_debug_inject_stall",
+           "mla_decode_noalloc", "mla_partial_grid", "mla_debug_inject_stall", "mla_debug_merge_plan",
            "mla_append_kv_fp8", "mla_rope_cos_sin_table", "mla_combine_f32",
            "mla_merge_rank_partials", "mla_fused_splits", "mla_fused_workspace_bytes",
            "mla_decode_fused",
@@ -107,6 +108,8 @@ def _load_lib():
     lib.mla_device_error_status.restype = i32
     lib.mla_debug_inject_stall.argtypes = [i32]
     lib.mla_debug_inject_stall.restype = i32
+    lib.mla_debug_merge_plan.argtypes = [i32, i32]
+    lib.mla_debug_merge_plan.restype = i32
     lib.mla_fused_splits.argtypes = [i32, i32, i32, i32]
     lib.mla_fused_splits.restype = i32
     lib.mla_fused_workspace_bytes.argtypes = [i32, i32, i32, i32]
@@ -390,6 +393,12 @@ def mla_debug_inject_stall(enable: bool) -> bool:
     their first CTA unissued, so its bounded waits run out and the kernel
     reports MLA_DEVERR_TIMEOUT.  Returns the previous setting."""
     return bool(_lib.mla_debug_inject_stall(1 if enable else 0))
+
+
+def mla_debug_merge_plan(v: int, gpi: int) -> None:
+    """Test hook: later single launches merge with v dims per thread and gpi
+    128-thread groups per item; (0, 0) restores the automatic choice."""
+    _check("mla_debug_merge_plan", _lib.mla_debug_merge_plan(int(v), int(gpi)))
 
 
 def decode(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits, max_splits,

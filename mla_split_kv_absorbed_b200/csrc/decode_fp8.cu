@@ -71,6 +71,7 @@
 // 384-511.
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.cuh"
 #include "mla.h"
@@ -345,7 +346,11 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
   auto write_empty = [&]() {
     for (int i = tid; i < rows_valid * 512; i += kThreads) {
       const int n = i >> 9;
-      args.part_o[((row_base + n) * slots + slot) * 512 + (i & 511)] = 0.0f;
+      const int64_t at = ((row_base + n) * slots + slot) * 512 + (i & 511);
+      if (args.fused)
+        args.part_o16[at] = 0;
+      else
+        args.part_o[at] = 0.0f;
     }
     if (tid < rows_valid) args.part_lse[(row_base + tid) * slots + slot] = -INFINITY;
   };
@@ -875,7 +880,8 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
         const bool nonempty = !bad && l > 0.0f;
         sc.m_run[n] = m_run;
         if (own) {
-          sc.inv_l[n] = nonempty ? args.kv_scale / l : 0.0f;
+          // the single launch keeps O in units of kv_scale (|O| <= 448 fits fp16)
+          sc.inv_l[n] = nonempty ? (args.fused ? 1.0f : args.kv_scale) / l : 0.0f;
           if (valid)
             args.part_lse[(row_base + n) * slots + slot] =
                 nonempty ? (m_run - kPShift + log2f(l)) * 0.69314718055994530942f : -INFINITY;
@@ -938,32 +944,54 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
   }
   if (warp >= 4) {
     // ============================================================ epilogue (warps 4-23)
-    // O^T / l -> part_o, the sixteen [128 dims x 16 rows] TMEM chunks
-    // spread over the five warpgroups (thread = latent dim of a block)
+    // O^T -> shared memory, the sixteen [128 dims x 16 rows] TMEM chunks
+    // spread over the five warpgroups (thread = latent dim of a block), as
+    // row-major [64 rows][512 dims] in the free ring: O/l (fp32, or fp16 in
+    // units of kv_scale in the single launch) when this CTA writes its own
+    // partial, which then leaves row by row in 16-byte stores; unnormalised
+    // fp32 O when the cut unit's pieces merge it across the cluster.
     tc_fence_after();
+    const int ewg = (warp - 4) >> 2;  // 0..4
+    const int wq = warp & 3;
+    const int d_lane = wq * 32 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+    float* staged = reinterpret_cast<float*>(smem + kOffRing);           // [64][512] fp32
+    uint16_t* staged_h = reinterpret_cast<uint16_t*>(smem + kOffRing);   // [64][512] fp16
     if (*abort_flag == 0) {
-      const int ewg = (warp - 4) >> 2;  // 0..4
-      const int wq = warp & 3;
-      const int d_lane = wq * 32 + lane;
-      const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-      float* po = args.part_o + (row_base * slots + slot) * 512;
-      const int64_t row_stride = (int64_t)slots * 512;
-      float* staged = reinterpret_cast<float*>(smem + kOffRing);  // [64][512], ring is free
 #pragma unroll 1
       for (int ch = ewg; ch < 16; ch += 5) {
         const int j = ch >> 2, grp = ch & 3;
         float v[16];
         tmem_ld16(t_lane + kTmemO + 64 * j + 16 * grp, v);
-        if (own) {
+        if (own && args.fused) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const int nn = grp * 16 + k;
-            if (nn < rows_valid) po[nn * row_stride + 128 * j + d_lane] = v[k] * sc.inv_l[nn];
+            staged_h[nn * 512 + 128 * j + d_lane] = __half_as_ushort(__float2half_rn(v[k] * sc.inv_l[nn]));
+          }
+        } else if (own) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int nn = grp * 16 + k;
+            staged[nn * 512 + 128 * j + d_lane] = v[k] * sc.inv_l[nn];
           }
         } else {
-          // unnormalised O, merged across the cluster below
 #pragma unroll
           for (int k = 0; k < 16; ++k) staged[(grp * 16 + k) * 512 + 128 * j + d_lane] = v[k];
+        }
+      }
+    }
+    if (own) {
+      named_bar_sync(6, kSoftThreads + 128);  // the staged rows are complete
+      if (*abort_flag == 0) {
+        const int vpr = args.fused ? 64 : 128;  // 16-byte vectors per row
+        const uint4* src = reinterpret_cast<const uint4*>(smem + kOffRing);
+        for (int i = tid - 128; i < rows_valid * vpr; i += kSoftThreads + 128) {
+          const int n = i / vpr, c = i - n * vpr;
+          const int64_t at = ((row_base + n) * slots + slot) * 512;
+          uint4* dst = args.fused ? reinterpret_cast<uint4*>(args.part_o16 + at)
+                                  : reinterpret_cast<uint4*>(args.part_o + at);
+          dst[c] = src[i];
         }
       }
     }
@@ -981,13 +1009,150 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
 
 // Single-launch mode, after every CTA's partial body: a grid barrier (the
 // launch is cooperative, so every CTA is resident), then the log-sum-exp
-// merge of each row's entries, spread over the grid: each 128-thread group
-// of a CTA merges one (row, 128-dim quarter) at a time, with all of a
-// thread's entry loads of a round issued before it accumulates, the split
-// weights from the entries' LSE, and sums in a fixed order (deterministic).
-// The last CTA to leave resets the two counters for the next launch.
+// merge of each row's entries, spread over the grid.  An item is a run of
+// 128 V dims of one row (thread t: dims t V .. t V + V - 1); gpi 128-thread
+// groups of one CTA share an item, group j taking entries j, j + gpi, ...;
+// a CTA works on 6 / gpi items at a time.  Each group merges its entries
+// against its own maximum LSE (every entry load of a batch issued before the
+// weights are applied), and the groups' results are combined through shared
+// memory, so every sum has a fixed order (deterministic).  Each batch's LSEs
+// are loaded with its values and folded into a running maximum, so a batch
+// costs one round trip to L2.  V and gpi are
+// chosen per launch by the launcher (merge_v, merge_gpi).  The last CTA to
+// leave resets the two counters for the next launch.
 constexpr int kMergeGroups = kThreads / 128;
-constexpr int kMergeBatch = 32;    // entry loads in flight per thread
+
+// The raw words of V consecutive fp16 entries, loaded as they are (one
+// register per entry for V <= 2, two for V = 4) and converted when used.
+template <int V>
+struct MergeRaw;
+template <>
+struct MergeRaw<1> {
+  using T = unsigned short;
+  __device__ static T load(const uint16_t* p) { return __ldcg(reinterpret_cast<const unsigned short*>(p)); }
+  __device__ static T zero() { return 0; }
+  __device__ static float at(T r, int) { return __half2float(__ushort_as_half(r)); }
+};
+template <>
+struct MergeRaw<2> {
+  using T = unsigned int;
+  __device__ static T load(const uint16_t* p) { return __ldcg(reinterpret_cast<const unsigned int*>(p)); }
+  __device__ static T zero() { return 0u; }
+  __device__ static float at(T r, int v) {
+    return __half2float(__ushort_as_half((unsigned short)(v ? r >> 16 : r & 0xFFFFu)));
+  }
+};
+template <>
+struct MergeRaw<4> {
+  using T = uint2;
+  __device__ static T load(const uint16_t* p) { return __ldcg(reinterpret_cast<const uint2*>(p)); }
+  __device__ static T zero() { return make_uint2(0u, 0u); }
+  __device__ static float at(T r, int v) {
+    const uint32_t w = v < 2 ? r.x : r.y;
+    return __half2float(__ushort_as_half((unsigned short)((v & 1) ? w >> 16 : w & 0xFFFFu)));
+  }
+};
+
+template <int V>
+__device__ __forceinline__ void merge_items(const DecodeArgs& a, uint8_t* smem) {
+  constexpr int kB = V == 4 ? 12 : 32;  // entries per batch: 24-32 registers of loads in flight
+  const int tid = threadIdx.x, grp = tid >> 7, t = tid & 127, lane = tid & 31;
+  const int gpi = a.merge_gpi, ipc = kMergeGroups / gpi;
+  const int sub = grp / gpi, j = grp % gpi;
+  const int chunks = 4 / V;
+  const int QH = a.q_len * a.H;
+  const int items = a.B * QH * chunks;
+  const int slots = a.max_splits * a.pieces;
+  // exchange: [sub][buffer][group][128 V acc | m | w], the ring is free
+  const int xstride = 128 * V + 2;
+  float* xbase = reinterpret_cast<float*>(smem + kOffRing) + sub * 2 * gpi * xstride;
+  int it = 0;
+  for (int item = (int)blockIdx.x + sub * (int)gridDim.x; item < items;
+       item += ipc * (int)gridDim.x, ++it) {
+    const int row = item / chunks, d = (item % chunks) * 128 * V + t * V;
+    const int bq = row / QH;
+    int S = a.splits_const > 0 ? a.splits_const : a.num_splits[bq];
+    S = S < 1 ? 0 : (S > a.max_splits ? a.max_splits : S);
+    const int E = S * a.pieces;
+    const int nj = E > j ? (E - j + gpi - 1) / gpi : 0;  // this group's entries
+    const uint16_t* po = a.part_o16 + (int64_t)row * slots * 512 + d;
+    const float* pl = a.part_lse + (int64_t)row * slots;
+    // the group's entries in batches of kB, each batch's LSEs loaded with its
+    // values (lane q: entry k0 + q), against a running maximum mj
+    float mj = -INFINITY, acc[V], wsum = 0.0f;
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+    for (int k0 = 0; k0 < nj; k0 += kB) {
+      typename MergeRaw<V>::T x[kB];
+#pragma unroll
+      for (int q = 0; q < kB; ++q)
+        x[q] = k0 + q < nj ? MergeRaw<V>::load(po + (int64_t)(j + gpi * (k0 + q)) * 512)
+                           : MergeRaw<V>::zero();
+      const float lq = (lane < kB && k0 + lane < nj) ? __ldcg(pl + j + gpi * (k0 + lane)) : -INFINITY;
+      float mb = lq;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+      if (mb > mj) {  // warp-uniform; the sums so far are rescaled to the new maximum
+        const float r = mj == -INFINITY ? 0.0f : expf(mj - mb);
+        wsum *= r;
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] *= r;
+        mj = mb;
+      }
+      const float wl = lq == -INFINITY ? 0.0f : expf(lq - mj);
+#pragma unroll
+      for (int q = 0; q < kB; ++q) {
+        const float w = __shfl_sync(0xffffffffu, wl, q);
+        wsum += w;
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = fmaf(w, MergeRaw<V>::at(x[q], v), acc[v]);
+      }
+    }
+    float M = mj, W = wsum;
+    if (gpi > 1) {
+      float* xb = xbase + (it & 1) * gpi * xstride;
+      float* mine = xb + j * xstride;
+#pragma unroll
+      for (int v = 0; v < V; ++v) mine[t * V + v] = acc[v];
+      if (t == 0) {
+        mine[128 * V] = mj;
+        mine[128 * V + 1] = wsum;
+      }
+      named_bar_sync(7 + sub, 128 * gpi);
+      if (j == 0) {
+        M = -INFINITY;
+        for (int g = 0; g < gpi; ++g) M = fmaxf(M, xb[g * xstride + 128 * V]);
+        W = 0.0f;
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+        for (int g = 0; g < gpi; ++g) {
+          const float mg = xb[g * xstride + 128 * V];
+          const float f = mg == -INFINITY ? 0.0f : expf(mg - M);
+          W = fmaf(f, xb[g * xstride + 128 * V + 1], W);
+#pragma unroll
+          for (int v = 0; v < V; ++v) acc[v] = fmaf(f, xb[g * xstride + t * V + v], acc[v]);
+        }
+      }
+    }
+    if (j == 0) {
+      const bool empty = M == -INFINITY || !(W > 0.0f);
+      const float f = empty ? 0.0f : a.kv_scale / W;  // the entries are in units of kv_scale
+      uint16_t h[V];
+#pragma unroll
+      for (int v = 0; v < V; ++v) h[v] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[v] * f));
+      uint16_t* dst = a.out + (int64_t)row * 512 + d;
+      if constexpr (V == 4) {
+        *reinterpret_cast<uint2*>(dst) =
+            make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+      } else if constexpr (V == 2) {
+        *reinterpret_cast<uint32_t*>(dst) = h[0] | ((uint32_t)h[1] << 16);
+      } else {
+        dst[0] = h[0];
+      }
+      if (a.out_lse != nullptr && d == 0) a.out_lse[row] = empty ? -INFINITY : M + logf(W);
+    }
+  }
+}
 
 __device__ __forceinline__ void fused_merge(const DecodeArgs& a, uint8_t* smem) {
   Scratch& sc = *reinterpret_cast<Scratch*>(smem + kOffScratch);
@@ -1010,62 +1175,12 @@ __device__ __forceinline__ void fused_merge(const DecodeArgs& a, uint8_t* smem) 
   }
   __syncthreads();
   if (sc.merge_fail == 0) {
-    const int grp = tid >> 7, t = tid & 127, lane = tid & 31, wid = t >> 5;
-    float* w_smem = reinterpret_cast<float*>(smem + kOffRing) + grp * 256;  // ring is free
-    float* red = reinterpret_cast<float*>(smem + kOffRing) + kMergeGroups * 256 + grp * 8;
-    const int QH = a.q_len * a.H;
-    const int rows = a.B * QH;
-    const int slots = a.max_splits * a.pieces;
-    for (int item = (int)blockIdx.x + grp * (int)gridDim.x; item < rows * 4;
-         item += kMergeGroups * (int)gridDim.x) {
-      const int row = item >> 2, d = (item & 3) * 128 + t;
-      const int bq = row / QH;
-      int S = a.splits_const > 0 ? a.splits_const : a.num_splits[bq];
-      S = S < 1 ? 0 : (S > a.max_splits ? a.max_splits : S);
-      const int E = S * a.pieces;  // entries of this row, at most 256
-      const float* po = a.part_o + (int64_t)row * slots * 512 + d;
-      const float* pl = a.part_lse + (int64_t)row * slots;
-      float v[kMergeBatch];
-#pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) v[j] = j < E ? __ldcg(po + (int64_t)j * 512) : 0.0f;
-      float lse[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) lse[k] = t + 128 * k < E ? __ldcg(pl + t + 128 * k) : -INFINITY;
-      float m = fmaxf(lse[0], lse[1]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      named_bar_sync(7 + grp, 128);  // red and w_smem of the previous item are no longer read
-      if (lane == 0) red[wid] = m;
-      named_bar_sync(7 + grp, 128);
-      m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      float wpart = 0.0f;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float w = lse[k] == -INFINITY ? 0.0f : expf(lse[k] - m);
-        if (t + 128 * k < E) w_smem[t + 128 * k] = w;
-        wpart += w;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wpart += __shfl_xor_sync(0xffffffffu, wpart, o);
-      if (lane == 0) red[4 + wid] = wpart;
-      named_bar_sync(7 + grp, 128);
-      const float wsum = (red[4] + red[5]) + (red[6] + red[7]);
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      for (int e0 = 0; e0 < E; e0 += kMergeBatch) {
-        if (e0 > 0) {
-#pragma unroll
-          for (int j = 0; j < kMergeBatch; ++j)
-            v[j] = e0 + j < E ? __ldcg(po + (int64_t)(e0 + j) * 512) : 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j)
-          if (e0 + j < E) acc[j & 3] = fmaf(w_smem[e0 + j], v[j], acc[j & 3]);
-      }
-      const float o = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      const bool empty = m == -INFINITY || !(wsum > 0.0f);
-      a.out[(int64_t)row * 512 + d] = __bfloat16_as_ushort(__float2bfloat16_rn(empty ? 0.0f : o / wsum));
-      if (a.out_lse != nullptr && (item & 3) == 0 && t == 0) a.out_lse[row] = empty ? -INFINITY : m + logf(wsum);
-    }
+    if (a.merge_v == 4)
+      merge_items<4>(a, smem);
+    else if (a.merge_v == 2)
+      merge_items<2>(a, smem);
+    else
+      merge_items<1>(a, smem);
   }
   __syncthreads();
   if (tid == 0 && atomicAdd(a.sync + 1, 1) == (int)gridDim.x - 1) {
@@ -1097,6 +1212,27 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map,
   const long long units = (long long)a.groups * a.max_splits * a.B;
   const long long ctas = a.split_from + a.pad + (units - a.split_from) * a.pieces;
   if (a.fused) {
+    // the merge plan: vector width V and groups per item with the fewest
+    // rounds of entry loads per CTA, (items per CTA slot) x (batches + 1)
+    DecodeArgs f = a;
+    const long long rows = (long long)a.B * a.q_len * a.H;
+    const int E = a.max_splits * a.pieces;
+    long long best = a.merge_v > 0 ? 0 : -1;  // a plan set by the test hook stands
+    for (int V : {4, 2, 1}) {
+      for (int gpi : {1, 2, 3, 6}) {
+        const long long items = rows * (4 / V);
+        const long long slots_per_round = ctas * (fp8k::kMergeGroups / gpi);
+        const long long per = (E + gpi - 1) / gpi;
+        const long long kb = V == 4 ? 12 : 32;  // entries per load batch
+        const long long cost =
+            ((items + slots_per_round - 1) / slots_per_round) * ((per + kb - 1) / kb + 1);
+        if (best < 0 || (a.merge_v == 0 && cost < best)) {
+          best = cost;
+          f.merge_v = V;
+          f.merge_gpi = gpi;
+        }
+      }
+    }
     // every CTA must be resident for the grid barrier: a cooperative launch
     // guarantees it (or fails), and the pieces need no cluster here
     cudaLaunchConfig_t cfg = {};
@@ -1109,7 +1245,7 @@ cudaError_t launch_decode_fp8(const DecodeArgs& a, const CUtensorMap& kv_map,
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fp8k::decode_fp8_kernel, a, kv_map, rope_map);
+    return cudaLaunchKernelEx(&cfg, fp8k::decode_fp8_kernel, f, kv_map, rope_map);
   }
   if (a.pieces == 1) {
     fp8k::decode_fp8_kernel<<<(unsigned)ctas, fp8k::kThreads, fp8k::kSmemBytes, stream>>>(a, kv_map,

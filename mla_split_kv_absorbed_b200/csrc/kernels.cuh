@@ -56,12 +56,16 @@ struct DecodeArgs {
   float q_scale;
   // Single-launch mode (FP8, every CTA resident, cooperative launch without
   // clusters): each piece writes its own normalised partial to entry
-  // s * pieces + piece of its rows (part_o / part_lse then hold
-  // max_splits * pieces entries per row), and after a grid barrier on
-  // sync[0] the grid merges them into out / out_lse; sync[1] counts the CTAs
-  // that have finished, and the last one resets both to zero.
+  // s * pieces + piece of its rows (part_o16 / part_lse then hold
+  // max_splits * pieces entries per row; O as fp16 in units of kv_scale,
+  // part_o is not used), and after a grid barrier on sync[0] the grid merges
+  // them into out / out_lse; sync[1] counts the CTAs that have finished, and
+  // the last one resets both to zero.
   int fused;
+  uint16_t* part_o16;   // [rows][entries][512] fp16, O / (l kv_scale)
   int splits_const;     // > 0: every request has this many splits (num_splits is not read)
+  int merge_v;          // single launch: dims per thread in the merge (1, 2 or 4)
+  int merge_gpi;        // single launch: 128-thread groups per merge item (1, 2, 3 or 6)
   uint16_t* out;        // [rows][512] bf16
   float* out_lse;       // [rows], may be null
   int32_t* sync;        // two counters, zero before the launch

@@ -16,6 +16,7 @@
 namespace {
 
 std::atomic<int> g_inject_stall{0};  // mla_debug_inject_stall
+std::atomic<int> g_merge_plan{0};    // mla_debug_merge_plan: 16 * V + gpi, 0 = automatic
 
 constexpr int kPage = 64;
 constexpr int kRow = 576;
@@ -192,6 +193,9 @@ int setup_decode(const uint16_t* q_nope, const uint16_t* q_rope, const void* kv_
   a->qk_scale_log2 = softmax_scale * kv_scale * 1.4426950408889634f;
   a->kv_scale = kv_scale;
   a->inject_stall = g_inject_stall.load(std::memory_order_relaxed);
+  const int plan_mv = g_merge_plan.load(std::memory_order_relaxed);
+  a->merge_v = plan_mv >> 4;  // 0: the launcher chooses
+  a->merge_gpi = plan_mv & 15;
   int32_t plan[4];
   plan_grid(B, q_len, H, max_splits, kv_dtype, num_sms_current_device(), plan);
   a->groups = (q_len * H + 63) / 64;
@@ -265,9 +269,10 @@ int fused_splits(int B, int q_len, int H, int num_sms) {
   return (int)(S > kFusedMaxEntries ? kFusedMaxEntries : S);
 }
 
+// counters, then the entries' O (fp16), then their LSE (fp32)
 size_t fused_bytes(int B, int q_len, int H, int S) {
   const size_t entries = (size_t)B * q_len * H * S;
-  return kFusedCounterBytes + entries * 512 * sizeof(float) + entries * sizeof(float);
+  return kFusedCounterBytes + entries * 512 * sizeof(uint16_t) + entries * sizeof(float);
 }
 
 }  // namespace
@@ -312,8 +317,9 @@ int mla_decode_fused(const uint16_t* q_nope, const uint16_t* q_rope, const void*
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.fused = 1;
   a.sync = reinterpret_cast<int32_t*>(ws);
-  a.part_o = reinterpret_cast<float*>(ws + kFusedCounterBytes);
-  a.part_lse = a.part_o + entries * 512;
+  a.part_o = nullptr;
+  a.part_o16 = reinterpret_cast<uint16_t*>(ws + kFusedCounterBytes);
+  a.part_lse = reinterpret_cast<float*>(a.part_o16 + entries * 512);
   a.out = out_bf16;
   a.out_lse = out_lse;
   return status_of(mla::launch_decode_fp8(a, map, rope_map, static_cast<cudaStream_t>(stream)));
@@ -442,6 +448,17 @@ int mla_partial_grid(int B, int q_len, int H, int max_splits, int kv_dtype, int 
 
 int mla_debug_inject_stall(int enable) {
   return g_inject_stall.exchange(enable != 0 ? 1 : 0, std::memory_order_relaxed);
+}
+
+int mla_debug_merge_plan(int v, int gpi) {
+  if (v == 0 && gpi == 0) {
+    g_merge_plan.store(0, std::memory_order_relaxed);
+    return MLA_OK;
+  }
+  if ((v != 1 && v != 2 && v != 4) || (gpi != 1 && gpi != 2 && gpi != 3 && gpi != 6))
+    return MLA_ERR_INVALID_ARG;
+  g_merge_plan.store(16 * v + gpi, std::memory_order_relaxed);
+  return MLA_OK;
 }
 
 }  // extern "C"

@@ -131,10 +131,11 @@ def test_fused_workspace_and_rejections_without_gpu(lib):
     assert h.mla_fused_splits(1, 1, 16, 1000) == 256
     assert h.mla_fused_splits(0, 1, 64, 148) == 0
     assert h.mla_fused_splits(1, 1, 64, 0) == 0
-    # counters (256 bytes) + O (512 fp32) and LSE per (row, split)
-    assert h.mla_fused_workspace_bytes(1, 1, 64, 148) == 256 + 64 * 148 * 513 * 4
-    assert h.mla_fused_workspace_bytes(16, 1, 64, 148) == 256 + 16 * 64 * 9 * 513 * 4
-    assert h.mla_fused_workspace_bytes(2, 4, 16, 148) == 256 + 2 * 4 * 16 * 74 * 513 * 4  # one row group
+    # counters (256 bytes) + O (512 fp16) and LSE (fp32) per (row, split)
+    per = 512 * 2 + 4
+    assert h.mla_fused_workspace_bytes(1, 1, 64, 148) == 256 + 64 * 148 * per
+    assert h.mla_fused_workspace_bytes(16, 1, 64, 148) == 256 + 16 * 64 * 9 * per
+    assert h.mla_fused_workspace_bytes(2, 4, 16, 148) == 256 + 2 * 4 * 16 * 74 * per  # one row group
     assert h.mla_fused_workspace_bytes(149, 1, 64, 148) == 0
     assert h.mla_fused_workspace_bytes(0, 1, 64, 148) == 0
     fake = ctypes.c_void_p(1 << 20)
@@ -153,6 +154,16 @@ def test_fused_workspace_and_rejections_without_gpu(lib):
     assert h.mla_decode_fused(*base, 1, 64, 1.0, fake, need - 1, fake, null, null, null) == lib.MLA_ERR_INVALID_ARG
     # the shared checks of mla_decode_partial apply
     assert h.mla_decode_fused(*base, 5, 64, 1.0, fake, big, fake, null, null, null) == lib.MLA_ERR_UNSUPPORTED
+
+
+def test_merge_plan_hook_without_gpu(lib):
+    h = lib.load()
+    for v, gpi in [(3, 1), (4, 4), (0, 1), (8, 6), (1, 0), (-1, 2)]:
+        assert h.mla_debug_merge_plan(v, gpi) == lib.MLA_ERR_INVALID_ARG
+    for v in (1, 2, 4):
+        for gpi in (1, 2, 3, 6):
+            assert h.mla_debug_merge_plan(v, gpi) == lib.MLA_OK
+    assert h.mla_debug_merge_plan(0, 0) == lib.MLA_OK
 
 
 def test_q8_rejections_without_gpu(lib):

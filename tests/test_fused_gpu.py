@@ -134,3 +134,30 @@ def test_fused_full_size_sampled_rows(spec):
     l = lse.cpu().numpy().reshape(R)[rows]
     assert_attention_close(o, l, o_ref, l_ref, what=spec + " fused")
     assert torch.count_nonzero(ws[:8]).item() == 0
+
+
+@pytest.mark.parametrize("spec,ov", [
+    ("b1_128k_fp8", dict(seq_lens=[64 * 148 * 2 + 5])),   # 148 entries per row
+    ("b16_128k_fp8", dict(seq_lens=[5000, 130, 1, 777])),  # 37 entries per row, empty rows' splits
+])
+def test_every_merge_plan_matches_the_oracle(spec, ov):
+    # the merge inside the single launch picks its plan from the shape; force
+    # each of the twelve (dims per thread, groups per item) plans in turn
+    import mla_split_kv_absorbed_b200 as m
+    c = make_case(spec, **ov)
+    w = c.w
+    rows = np.arange(w.B * w.q_len * w.H)
+    o_ref, l_ref = oracle_rows(c, rows)
+    ws = m.alloc_fused_workspace(w.B, w.q_len, w.H)
+    try:
+        for v in (1, 2, 4):
+            for gpi in (1, 2, 3, 6):
+                m.mla_debug_merge_plan(v, gpi)
+                out, lse, err, _ = run_fused(c, workspace=ws)
+                assert err == 0
+                assert_attention_close(out.float().cpu().numpy().reshape(-1, 512),
+                                       lse.cpu().numpy().reshape(-1), o_ref, l_ref,
+                                       what=f"{spec} plan v={v} gpi={gpi}")
+                assert torch.count_nonzero(ws[:8]).item() == 0
+    finally:
+        m.mla_debug_merge_plan(0, 0)
