@@ -272,39 +272,34 @@ def run_single_launch(w, kv, steps, warmup, flush_bytes=256 << 20):
 
 
 def run_e2e(w, kv, steps, warmup, fused):
-    """Same step through the public API with host buffers: per step, pinned-host
-    -> device copies of the step's inputs (queries, seq_lens, block table, and
-    num_splits for the two-kernel step), the decode call, and device -> host
-    copies of O and LSE.  The KV cache stays resident in HBM, as in serving."""
+    """Same step through the public API with host buffers: per step, one
+    pinned-host -> device copy of the step's inputs (queries, seq_lens, block
+    table, and num_splits for the two-kernel step, packed by HostStaging), the
+    decode call, and one device -> host copy of O and LSE.  The KV cache stays
+    resident in HBM, as in serving."""
     import torch
     import mla_split_kv_absorbed_b200 as m
     stream = torch.cuda.current_stream()
-    src = [w.q_nope, w.q_rope, w.seq_lens, w.block_table] + ([] if fused else [w.num_splits])
-    h_in = [t.cpu().pin_memory() for t in src]
-    d_in = [torch.empty_like(t, device="cuda") for t in h_in]
+    st = m.HostStaging(w.B, w.q_len, w.H, w.block_table.shape[1], with_num_splits=not fused)
+    for name in st.host:
+        st.host[name].copy_(getattr(w, name).cpu())
     if fused:
         fws = m.alloc_fused_workspace(w.B, w.q_len, w.H)
     else:
         part = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
-    out = torch.empty((w.B, w.q_len, w.H, 512), dtype=torch.bfloat16, device="cuda")
-    out_lse = torch.empty((w.B, w.q_len, w.H), dtype=torch.float32, device="cuda")
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(out_lse.shape, dtype=out_lse.dtype).pin_memory()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    h2d = sum(t.numel() * t.element_size() for t in h_in)
-    d2h = out.numel() * 2 + out_lse.numel() * 4
+    d = st.dev
 
     def step():
-        for h, d in zip(h_in, d_in):
-            d.copy_(h, non_blocking=True)
+        st.upload(stream)
         if fused:
-            m.mla_decode_fused(d_in[0], d_in[1], kv, w.kv_scale, d_in[3], d_in[2],
-                               w.softmax_scale, fws, out, out_lse)
+            m.mla_decode_fused(d["q_nope"], d["q_rope"], kv, w.kv_scale, d["block_table"],
+                               d["seq_lens"], w.softmax_scale, fws, st.out, st.out_lse)
         else:
-            m.decode(d_in[0], d_in[1], kv, w.kv_scale, d_in[3], d_in[2], d_in[4], w.max_splits,
-                     w.softmax_scale, out=out, out_lse=out_lse, workspace=part)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(out_lse, non_blocking=True)
+            m.decode(d["q_nope"], d["q_rope"], kv, w.kv_scale, d["block_table"], d["seq_lens"],
+                     d["num_splits"], w.max_splits, w.softmax_scale, out=st.out,
+                     out_lse=st.out_lse, workspace=part)
+        st.download(stream)
 
     for _ in range(warmup):
         flush.zero_()
@@ -319,7 +314,7 @@ def run_e2e(w, kv, steps, warmup, fused):
         e1.record(stream)
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1) * 1e-3)
-    return statistics.median(times), h2d, d2h
+    return statistics.median(times), st.in_bytes, st.out_bytes
 
 
 def cpu_model():

@@ -24,6 +24,8 @@ Entry points (same names as the C ABI):
 * ``mla_device_error_status(word)`` / ``check_device_error(dev_error)`` — fold
   the GPU's error word into MLA_ERR_DEVICE.
 * ``mla_partial_grid(...)`` — host helper: the partial kernel's CTA layout for a shape.
+* ``HostStaging`` — one pinned host buffer and one copy each way for a step's
+  inputs and outputs (the host-buffer path).
 * ``mla_debug_inject_stall(enable)`` — test hook for the bounded-wait failure path.
 * ``mla_debug_merge_plan(v, gpi)`` — test hook: force the single launch's merge plan.
 
@@ -399,6 +401,61 @@ def mla_debug_merge_plan(v: int, gpi: int) -> None:
     """Test hook: later single launches merge with v dims per thread and gpi
     128-thread groups per item; (0, 0) restores the automatic choice."""
     _check("mla_debug_merge_plan", _lib.mla_debug_merge_plan(int(v), int(gpi)))
+
+
+class HostStaging:
+    """Host <-> device staging for one decode shape: a step's inputs (q_nope,
+    q_rope, seq_lens, block_table and, optionally, num_splits) live in one
+    pinned host buffer and go to the device in one copy; the outputs (O bf16
+    and LSE fp32) come back in one copy.  Fill the host views (``host[name]``)
+    and call ``upload()``; pass the device views (``dev[name]``) and
+    ``out`` / ``out_lse`` to the decode call; ``download()`` copies the outputs
+    into ``host_out`` / ``host_lse``.  Only torch copies: plumbing."""
+
+    _ALIGN = 256
+
+    def __init__(self, B, q_len, H, max_pages, with_num_splits=False, device="cuda"):
+        spec = [("q_nope", torch.bfloat16, (B, q_len, H, 512)),
+                ("q_rope", torch.bfloat16, (B, q_len, H, 64)),
+                ("seq_lens", torch.int32, (B,)),
+                ("block_table", torch.int32, (B, max_pages))]
+        if with_num_splits:
+            spec.append(("num_splits", torch.int32, (B,)))
+        self.h_in, self.d_in, self.host, self.dev = self._carve(spec, device)
+        self.in_bytes = self.h_in.numel()
+        out_spec = [("out", torch.bfloat16, (B, q_len, H, 512)),
+                    ("out_lse", torch.float32, (B, q_len, H))]
+        self.h_out, self.d_out, hviews, dviews = self._carve(out_spec, device)
+        self.out_bytes = self.h_out.numel()
+        self.out, self.out_lse = dviews["out"], dviews["out_lse"]
+        self.host_out, self.host_lse = hviews["out"], hviews["out_lse"]
+
+    @classmethod
+    def _carve(cls, spec, device):
+        offs, n = [], 0
+        for _, dt, shape in spec:
+            nbytes = torch.empty((), dtype=dt).element_size()
+            for d in shape:
+                nbytes *= d
+            offs.append((n, nbytes))
+            n += (nbytes + cls._ALIGN - 1) // cls._ALIGN * cls._ALIGN
+        h = torch.empty(n, dtype=torch.uint8).pin_memory()
+        d = torch.empty(n, dtype=torch.uint8, device=device)
+        hv, dv = {}, {}
+        for (name, dt, shape), (o, nb) in zip(spec, offs):
+            hv[name] = h[o:o + nb].view(dt).view(shape)
+            dv[name] = d[o:o + nb].view(dt).view(shape)
+        return h, d, hv, dv
+
+    def upload(self, stream=None):
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            self.d_in.copy_(self.h_in, non_blocking=True)
+
+    def download(self, stream=None):
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            self.h_out.copy_(self.d_out, non_blocking=True)
 
 
 def decode(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits, max_splits,

@@ -161,3 +161,26 @@ def test_every_merge_plan_matches_the_oracle(spec, ov):
                 assert torch.count_nonzero(ws[:8]).item() == 0
     finally:
         m.mla_debug_merge_plan(0, 0)
+
+
+def test_host_staging_round_trip_matches_device_inputs():
+    # one packed host-to-device copy of the inputs, one device-to-host copy of
+    # the outputs: the same bits as the call on device-resident inputs
+    import mla_split_kv_absorbed_b200 as m
+    c = make_case("b16_128k_fp8", seq_lens=[3000, 700, 64])
+    w = c.w
+    st = m.HostStaging(w.B, w.q_len, w.H, w.block_table.shape[1])
+    for name in st.host:
+        st.host[name].copy_(getattr(w, name).cpu())
+    ws = m.alloc_fused_workspace(w.B, w.q_len, w.H)
+    st.upload()
+    d = st.dev
+    m.mla_decode_fused(d["q_nope"], d["q_rope"], c.kv_dev, w.kv_scale, d["block_table"],
+                       d["seq_lens"], w.softmax_scale, ws, st.out, st.out_lse)
+    st.download()
+    torch.cuda.synchronize()
+    out, lse, err, _ = run_fused(c)
+    assert err == 0
+    assert torch.equal(st.host_out.view(torch.int16), out.cpu().view(torch.int16))
+    assert torch.equal(st.host_lse, lse.cpu())
+    assert st.in_bytes >= (w.q_nope.numel() + w.q_rope.numel()) * 2 + w.block_table.numel() * 4
