@@ -474,7 +474,10 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
         ++win;
         win_hi = load_window(win + 1);
       }
-      prefetch_tile(i);
+      // with several query-row groups the split's CTAs read the same pages
+      // (the first reader brings them into L2) and the prefetches only add
+      // to the queues: measured 2.4% faster at q_len 4 without them
+      if (args.groups == 1) prefetch_tile(i);
       const int tok0 = t0 + i * kTile;
       const int pa = page_at(2 * i);
       const bool want_b = tok0 + 64 < t1;
