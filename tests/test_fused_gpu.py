@@ -118,17 +118,20 @@ def test_fused_refuses_shapes_without_a_single_wave_and_small_workspaces():
     assert e.value.status == m.MLA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("spec", ["b1_128k_fp8", "b16_128k_fp8"])
+@pytest.mark.parametrize("spec", ["b1_128k_fp8", "b16_128k_fp8", "verify_q4_256k_fp8"])
 def test_fused_full_size_sampled_rows(spec):
     # the benchmark workloads at full size, in the launch the benchmark times
-    # (batch 1: 148 splits; batch 16: 9 splits, 144 CTAs on 148 SMs)
+    # (batch 1: 148 splits; batch 16: 9 splits, 144 CTAs; the q_len-4 verify at
+    # batch 8: 4 row groups x 4 splits x 8 requests, 128 CTAs); one sampled
+    # row of every (request, query position), both ends, and random extras
     c = make_case(spec, gen_device="cuda")
     w = c.w
     out, lse, err, ws = run_fused(c)
     assert err == 0
     R = w.B * w.q_len * w.H
     rng = np.random.default_rng(7)
-    rows = np.unique(np.concatenate([[0, R - 1], rng.choice(R, size=24, replace=False)]))
+    per = [(b * w.q_len + q) * w.H + int(rng.integers(w.H)) for b in range(w.B) for q in range(w.q_len)]
+    rows = np.unique(np.concatenate([[0, R - 1], per, rng.choice(R, size=8, replace=False)]))
     o_ref, l_ref = oracle_rows(c, rows)
     o = out.float().cpu().numpy().reshape(R, 512)[rows]
     l = lse.cpu().numpy().reshape(R)[rows]
