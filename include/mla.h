@@ -296,14 +296,16 @@ MLA_API int mla_rope_cos_sin_table(float* cos_sin_host, int64_t max_pos, double 
 
 /* Host helper (article bullet "64 路 split-KV": batch-1 decode needs enough
  * splits to occupy the SMs; the pages fix no rule, so this is a reading):
- * one split per 2048 tokens of each request,
- *   out_host[b] = min(max_splits, max(1, ceil(seq_lens_host[b] / 2048))),
- * which gives 64 splits for a 128K-token request.  The rule itself does not
- * depend on num_sms: when the resulting grid underfills the GPU,
- * mla_decode_partial cuts each split across a CTA cluster on its own (see
- * mla_partial_grid).  num_sms (the target's SM count, > 0) is validated only.
- * seq_lens_host and out_host are HOST arrays of B int32; every seq_len must
- * be >= 1.  Returns MLA_ERR_INVALID_ARG for null pointers or sizes <= 0. */
+ * a batch's tokens are cut into at most about num_sms splits of equal length,
+ *   T = max(2048, ceil(sum_b seq_lens_host[b] / max(1, num_sms - B))) tokens,
+ *   out_host[b] = min(max_splits, max(1, ceil(seq_lens_host[b] / T))),
+ * so that no split is longer than T and, for B < num_sms, the batch has at
+ * most num_sms splits.  A single 128K-token request gets 64 splits (T =
+ * 2048); 16 such requests on 148 SMs get 9 each (one wave).  When the grid
+ * still underfills the GPU, mla_decode_partial cuts each split across a CTA
+ * cluster on its own (see mla_partial_grid).  seq_lens_host and out_host are
+ * HOST arrays of B int32; every seq_len must be >= 1.  Returns
+ * MLA_ERR_INVALID_ARG for null pointers, sizes <= 0 or num_sms <= 0. */
 MLA_API int mla_choose_splits(const int32_t* seq_lens_host, int B, int num_sms, int max_splits,
                               int32_t* out_host);
 

@@ -20,7 +20,7 @@ std::atomic<int> g_merge_plan{0};    // mla_debug_merge_plan: 16 * V + gpi, 0 = 
 
 constexpr int kPage = 64;
 constexpr int kRow = 576;
-constexpr int kSplitTokens = 2048;  // mla_choose_splits: tokens per split
+constexpr int kSplitTokens = 2048;  // mla_choose_splits: the fewest tokens per split
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -365,9 +365,16 @@ int mla_choose_splits(const int32_t* seq_lens_host, int B, int num_sms, int max_
     return MLA_ERR_INVALID_ARG;
   for (int b = 0; b < B; ++b)
     if (seq_lens_host[b] < 1) return MLA_ERR_INVALID_ARG;
-  // one split per 2048 tokens (32 pages), at least one, at most max_splits
+  // T = max(2048, ceil(sum_b L_b / max(1, num_sms - B))) tokens per split,
+  // and every request gets ceil(L_b / T) splits, at least one, at most
+  // max_splits: sum_b ceil(L_b / T) <= sum_b L_b / T + B <= num_sms
+  int64_t total = 0;
+  for (int b = 0; b < B; ++b) total += seq_lens_host[b];
+  const int64_t slots = num_sms - B > 1 ? num_sms - B : 1;
+  int64_t T = (total + slots - 1) / slots;
+  if (T < kSplitTokens) T = kSplitTokens;
   for (int b = 0; b < B; ++b) {
-    int64_t sp = ((int64_t)seq_lens_host[b] + kSplitTokens - 1) / kSplitTokens;
+    int64_t sp = ((int64_t)seq_lens_host[b] + T - 1) / T;
     if (sp < 1) sp = 1;
     if (sp > max_splits) sp = max_splits;
     out_host[b] = (int32_t)sp;

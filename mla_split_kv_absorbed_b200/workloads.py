@@ -56,9 +56,12 @@ class Spec:
     spare_pages: int = 4
 
 
-def splits_by_length(L: int, max_splits: int = 64) -> int:
-    """Per-request split count for ragged batches: one split per 2048 tokens, 1..64."""
-    return max(1, min(max_splits, -(-L // 2048)))
+def splits_by_length(lens, num_sms: int = 148, max_splits: int = 64):
+    """Per-request split counts for a ragged batch: splits of at most
+    T = max(2048, ceil(sum(lens) / max(1, num_sms - B))) tokens, ceil(L / T)
+    per request, 1..max_splits (at most num_sms splits when B < num_sms)."""
+    T = max(2048, -(-sum(int(L) for L in lens) // max(1, num_sms - len(lens))))
+    return [max(1, min(max_splits, -(-int(L) // T))) for L in lens]
 
 
 SPECS = {
@@ -154,7 +157,7 @@ def make(spec, device="cpu", seq_lens=None, B=None, H=None, q_len=None, splits=N
     assert len(lens) == Bn and all(L >= Q for L in lens)
 
     if spec.splits == "by_length":
-        nsp = [splits_by_length(L) for L in lens]
+        nsp = splits_by_length(lens)
     else:
         nsp = [int(spec.splits)] * Bn
     max_splits = max(nsp)

@@ -59,22 +59,28 @@ def test_status_strings(lib):
 
 
 def test_choose_splits_follows_the_length_rule(lib):
-    # the reading the ragged workload uses: one split per 2048 tokens, 1..max_splits
+    # the reading the ragged workload uses: about num_sms equal splits per batch
     from mla_split_kv_absorbed_b200 import workloads as wl
     rng = np.random.default_rng(7)
-    lens = np.concatenate([[1, 2047, 2048, 2049, 4096, 131072, 262144, 1 << 30],
+    lens = np.concatenate([[1, 2047, 2048, 2049, 4096, 131072, 262144],
                            rng.integers(1, 300000, size=500)]).astype(np.int32)
-    got = lib.mla_choose_splits(lens, 148, 64).numpy()
-    want = np.array([wl.splits_by_length(int(L)) for L in lens])
-    assert np.array_equal(got, want)
-    # the formula itself, written out: ceil(L / 2048) clamped to [1, max_splits]
-    for max_splits in (1, 7, 64, 256):
-        got = lib.mla_choose_splits(lens, 148, max_splits).numpy()
-        assert np.array_equal(got, np.clip(-(-lens.astype(np.int64) // 2048), 1, max_splits))
+    for sms in (1, 148, 1000):
+        got = lib.mla_choose_splits(lens, sms, 64).numpy()
+        assert np.array_equal(got, np.array(wl.splits_by_length(lens.tolist(), sms, 64)))
+    # the formula written out: T = max(2048, ceil(sum / max(1, SMs - B))), ceil(L / T) in [1, max]
+    L64 = lens.astype(np.int64)
+    for sms, max_splits in ((148, 64), (148, 7), (1000, 256), (1, 1)):
+        T = max(2048, -(-int(L64.sum()) // max(1, sms - len(lens))))
+        want = np.clip(-(-L64 // T), 1, max_splits)
+        assert np.array_equal(lib.mla_choose_splits(lens, sms, max_splits).numpy(), want)
     assert lib.mla_choose_splits([131072], 148, 64).tolist() == [64]  # the batch-1 64-way split
-    # the SM count does not change the rule
-    assert np.array_equal(lib.mla_choose_splits(lens, 1, 64).numpy(),
-                          lib.mla_choose_splits(lens, 148, 64).numpy())
+    assert lib.mla_choose_splits([131072] * 16, 148, 64).tolist() == [9] * 16  # one wave
+    assert lib.mla_choose_splits([1024], 148, 64).tolist() == [1]
+    # at most num_sms splits (one wave at one row group) for a batch of B < SMs
+    for _ in range(20):
+        big = rng.integers(1, 262145, size=int(rng.integers(1, 100))).astype(np.int32)
+        n = int(lib.mla_choose_splits(big, 148, 256).sum())
+        assert n <= 148 or int(big.sum()) <= 2048 * len(big)
     with pytest.raises(lib.MlaError):
         lib.mla_choose_splits([0], 148, 64)  # empty request
     with pytest.raises(lib.MlaError):
