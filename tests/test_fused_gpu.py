@@ -23,6 +23,11 @@ SMALL = [
     ("verify_q4_256k_fp8", dict(seq_lens=[777], H=16)),     # q_len 4, causal, one row group
     ("verify_q4_256k_fp8", dict(seq_lens=[1000, 4])),       # four row groups, 18 splits
     ("b16_128k_fp8", dict(seq_lens=[300] * 148)),           # one split per request
+    ("b16_128k_fp8", dict(seq_lens=[1024], H=16)),          # 16 rows in a 64-row group
+    ("b16_128k_fp8", dict(seq_lens=[3000], H=128)),         # two row groups, 74 splits
+    ("b16_128k_fp8", dict(seq_lens=[1500, 900], H=32, q_len=2)),  # causal, 2 positions per group
+    ("b16_128k_fp8", dict(seq_lens=[700, 5, 2200], H=16, q_len=3)),  # 48 rows, q_len 3
+    ("b16_128k_fp8", dict(seq_lens=[130, 64, 1, 2000] * 25)),  # 100 requests, 1 split each
 ]
 
 
