@@ -275,8 +275,9 @@ def run_e2e(w, kv, steps, warmup, fused):
     """Same step through the public API with host buffers: per step, one
     pinned-host -> device copy of the step's inputs (queries, seq_lens, block
     table, and num_splits for the two-kernel step, packed by HostStaging), the
-    decode call, and one device -> host copy of O and LSE.  The KV cache stays
-    resident in HBM, as in serving."""
+    decode call, and one device -> host copy of O and LSE; for the single
+    launch the three are one CUDA graph (DecodeGraph), replayed every step.
+    The KV cache stays resident in HBM, as in serving."""
     import torch
     import mla_split_kv_absorbed_b200 as m
     stream = torch.cuda.current_stream()
@@ -284,21 +285,20 @@ def run_e2e(w, kv, steps, warmup, fused):
     for name in st.host:
         st.host[name].copy_(getattr(w, name).cpu())
     if fused:
-        fws = m.alloc_fused_workspace(w.B, w.q_len, w.H)
+        graph = m.DecodeGraph(st, kv, w.kv_scale, w.softmax_scale)
     else:
         part = m.alloc_partials(w.B, w.q_len, w.H, w.max_splits)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     d = st.dev
 
     def step():
-        st.upload(stream)
         if fused:
-            m.mla_decode_fused(d["q_nope"], d["q_rope"], kv, w.kv_scale, d["block_table"],
-                               d["seq_lens"], w.softmax_scale, fws, st.out, st.out_lse)
-        else:
-            m.decode(d["q_nope"], d["q_rope"], kv, w.kv_scale, d["block_table"], d["seq_lens"],
-                     d["num_splits"], w.max_splits, w.softmax_scale, out=st.out,
-                     out_lse=st.out_lse, workspace=part)
+            graph.replay(stream)
+            return
+        st.upload(stream)
+        m.decode(d["q_nope"], d["q_rope"], kv, w.kv_scale, d["block_table"], d["seq_lens"],
+                 d["num_splits"], w.max_splits, w.softmax_scale, out=st.out,
+                 out_lse=st.out_lse, workspace=part)
         st.download(stream)
 
     for _ in range(warmup):

@@ -25,7 +25,8 @@ Entry points (same names as the C ABI):
   the GPU's error word into MLA_ERR_DEVICE.
 * ``mla_partial_grid(...)`` — host helper: the partial kernel's CTA layout for a shape.
 * ``HostStaging`` — one pinned host buffer and one copy each way for a step's
-  inputs and outputs (the host-buffer path).
+  inputs and outputs (the host-buffer path); ``DecodeGraph`` — that step with
+  the single launch captured as one CUDA graph.
 * ``mla_debug_inject_stall(enable)`` — test hook for the bounded-wait failure path.
 * ``mla_debug_merge_plan(v, gpi)`` — test hook: force the single launch's merge plan.
 
@@ -456,6 +457,45 @@ class HostStaging:
         s = torch.cuda.current_stream() if stream is None else stream
         with torch.cuda.stream(s):
             self.h_out.copy_(self.d_out, non_blocking=True)
+
+
+class DecodeGraph:
+    """One decode step over host buffers captured as a CUDA graph: the
+    HostStaging upload, the single launch (mla_decode_fused) and the download,
+    replayed with one call, so the three need no host launches between them.
+    The graph reads the staging buffers, the KV pool and the workspace at
+    replay time: fill ``staging.host`` and call ``replay()``; the outputs land
+    in ``staging.host_out`` / ``staging.host_lse`` once the stream reaches the
+    end of the replay."""
+
+    def __init__(self, staging, kv_pages, kv_scale, softmax_scale, workspace=None,
+                 dev_error=None, warmup=2):
+        self.st = staging
+        d = staging.dev
+        B, q_len, H, _ = d["q_nope"].shape
+        self.workspace = alloc_fused_workspace(B, q_len, H) if workspace is None else workspace
+        self.stream = torch.cuda.Stream()
+        self.graph = torch.cuda.CUDAGraph()
+        args = (d["q_nope"], d["q_rope"], kv_pages, kv_scale, d["block_table"], d["seq_lens"],
+                softmax_scale, self.workspace, staging.out, staging.out_lse, dev_error)
+
+        def step():
+            staging.upload(self.stream)
+            mla_decode_fused(*args, stream=self.stream)
+            staging.download(self.stream)
+        self.stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                step()
+        self.stream.synchronize()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            step()
+        self.stream.synchronize()
+
+    def replay(self, stream=None):
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            self.graph.replay()
 
 
 def decode(q_nope, q_rope, kv_pages, kv_scale, block_table, seq_lens, num_splits, max_splits,

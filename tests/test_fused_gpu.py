@@ -192,3 +192,33 @@ def test_host_staging_round_trip_matches_device_inputs():
     assert torch.equal(st.host_out.view(torch.int16), out.cpu().view(torch.int16))
     assert torch.equal(st.host_lse, lse.cpu())
     assert st.in_bytes >= (w.q_nope.numel() + w.q_rope.numel()) * 2 + w.block_table.numel() * 4
+
+
+def test_decode_graph_replays_the_host_buffer_step():
+    # the captured step (upload, single launch, download) gives the same bits
+    # as the call on device-resident inputs, and follows new host inputs
+    import mla_split_kv_absorbed_b200 as m
+    c = make_case("b16_128k_fp8", seq_lens=[3000, 700, 64])
+    w = c.w
+    st = m.HostStaging(w.B, w.q_len, w.H, w.block_table.shape[1])
+    for name in st.host:
+        st.host[name].copy_(getattr(w, name).cpu())
+    g = m.DecodeGraph(st, c.kv_dev, w.kv_scale, w.softmax_scale)
+    st.host_out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    out, lse, err, _ = run_fused(c)
+    assert err == 0
+    assert torch.equal(st.host_out.view(torch.int16), out.cpu().view(torch.int16))
+    assert torch.equal(st.host_lse, lse.cpu())
+    # new queries in the same host buffer: the next replay uses them
+    st.host["q_nope"].mul_(-1)
+    st.host["q_rope"].mul_(-1)
+    g.replay()
+    torch.cuda.synchronize()
+    c.dev["q_nope"].mul_(-1)
+    c.dev["q_rope"].mul_(-1)
+    out2, lse2, err2, _ = run_fused(c)
+    assert err2 == 0
+    assert torch.equal(st.host_out.view(torch.int16), out2.cpu().view(torch.int16))
+    assert not torch.equal(out2.view(torch.int16), out.view(torch.int16))
