@@ -89,7 +89,8 @@ constexpr int kChunk = 128 * 64;    // 128 tokens x 64 dims of E4M3 = 8 KiB
 constexpr int kPair = 2 * kChunk;   // 128 latent dims of a tile
 constexpr int kRingPairs = 11;      // latent pair slots: 2.75 tiles in flight
 constexpr int kRopeSlots = 1;      // freed by its tile's QK, refilled first for the next tile
-constexpr int kPBufs = 2;          // P buffers: the softmax of tile i+1 need not wait for PV(i)
+constexpr int kPBufs = 2;          // P buffers (1 or 2): with 2 the softmax of tile i+1 need not wait for PV(i)
+static_assert(kPBufs == 1 || kPBufs == 2, "the alpha and PV-done handshakes assume at most 2");
 constexpr float kPShift = 4.0f;     // log2 of the factor carried by the softmax weights
 constexpr float kLazy = 4.75f;      // the used max moves only when exceeded by more than this
 
@@ -601,10 +602,10 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
         }
       }
       // ---------------- O^T += V(np)^T . (P_hi + P_lo), after any QK that was ready
-      if (np < nq && ready(kBarPFull + (np & 1), (np >> 1) & 1) &&
+      if (np < nq && ready(kBarPFull + np % kPBufs, (np / kPBufs) & 1) &&
           ready(kBarOReady + (np & 1), (np >> 1) & 1)) {
         tc_fence_after();
-        const uint64_t dPhi = desc_at(dP, (np & 1) * 2 * kChunk), dPlo = desc_at(dPhi, kChunk);
+        const uint64_t dPhi = desc_at(dP, (np % kPBufs) * 2 * kChunk), dPlo = desc_at(dPhi, kChunk);
         // block by block, so each latent pair can be refilled as soon as its
         // block is done
 #pragma unroll
@@ -620,7 +621,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
           // latent pair j of this tile is free once its block's MMAs complete
           umma_commit_elect(&bars[kBarEmpty + slot]);
         }
-        umma_commit_elect(&bars[kBarPEmpty + (np & 1)]);
+        umma_commit_elect(&bars[kBarPEmpty + np % kPBufs]);
         umma_commit_elect(&bars[kBarPvDone]);
         if (np == T - 1) umma_commit_elect(&bars[kBarPvAll]);
         ++np;
@@ -830,11 +831,12 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
           m_run = tm;
         }
       }
-      // P buffer i % 2 free: PV of tile i - 2 done.  Waited for before this
-      // tile's alpha goes out: PV(i - 2) waited for the rescale of tile i - 2,
-      // so that alpha slot has been read, and the PV-done count the rescale
-      // warps test is at least i - 1.
-      if (i >= kPBufs) bad |= !mbar_wait(&bars[kBarPEmpty + (i & 1)], ((i >> 1) - 1) & 1, abort_flag);
+      // P buffer i % kPBufs free: PV of tile i - kPBufs done.  Waited for
+      // before this tile's alpha goes out: PV(i - kPBufs) waited for the
+      // rescale of that tile, so the alpha slot i % 2 has been read, and the
+      // PV-done count the rescale warps test is at least i - 1.
+      if (i >= kPBufs)
+        bad |= !mbar_wait(&bars[kBarPEmpty + i % kPBufs], ((i / kPBufs) - 1) & 1, abort_flag);
       // the rescale warps learn, per tile, which rows moved and by how much
       if (c == 0) {
         const uint32_t mask = __ballot_sync(0xffffffffu, moved && part == 0);
@@ -854,7 +856,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
       l_run = fmaf(l_run, alpha, psum);
       uint4 phi, plo;
       split16(pv, phi, plo);
-      const uint32_t p_off = kOffP + (i & 1) * 2 * kChunk + sw128(n, 32 * c + 16 * part);
+      const uint32_t p_off = kOffP + (i % kPBufs) * 2 * kChunk + sw128(n, 32 * c + 16 * part);
       *reinterpret_cast<uint4*>(smem + p_off) = phi;
       *reinterpret_cast<uint4*>(smem + p_off + kChunk) = plo;
       if (t0 + i * kTile + kTile > t1) {
@@ -870,7 +872,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarPFull + (i & 1)]);
+      if (lane == 0) mbar_arrive(&bars[kBarPFull + i % kPBufs]);
     }
     // ---- row sums: reduce l over the 8 threads of row n, in a fixed order
     {
