@@ -20,11 +20,11 @@
 // operands E4M3.  Q (bf16, 8 significant bits) is scaled per row by a power
 // of two and split as Q = Q_hi + Q_lo with Q_hi = Q rounded to 4 significant
 // bits and Q_lo = E4M3(Q - Q_hi); this is exact for every element within a
-// factor 2^-9 of the row maximum.  The softmax weights are scaled by 2^4,
-// p' = 2^(s - m + 4), and split the same way, P = P_hi + P_lo: about 8
+// factor 2^-9 of the row maximum.  The softmax weights are scaled by 2^3.5,
+// p' = 2^(s - m + 3.5), and split the same way, P = P_hi + P_lo: about 8
 // significant bits (like bf16) for every p' >= 2^-1 and an absolute error of
 // at most 2^-10 for smaller weights, while the largest weight of a row is at
-// least 2^4.  The scale cancels in O / l and is removed from the LSE.
+// least 2^3.5.  The scale cancels in O / l and is removed from the LSE.
 //
 // Tensor-core mapping.  QK^T takes the 128 two-term query rows as M and the
 // 128 tokens of a tile as N:
@@ -46,7 +46,7 @@
 //
 // Online softmax (log2 domain, scores pre-multiplied by log2 e), with a lazy
 // running max: the max m used for a row only moves when a tile's max exceeds
-// it by more than 4.75 (log2 units), so p' stays <= 2^8.75 < 448, the E4M3
+// it by more than 5.25 (log2 units), so p' stays <= 2^8.75 < 448, the E4M3
 // maximum.  A tile in which no score of a quadrant's rows exceeds its max by
 // that much (the common case once the max has settled) skips the max
 // reduction altogether: one barrier vote decides it.  O^T columns and row
@@ -91,8 +91,9 @@ constexpr int kRingPairs = 11;      // latent pair slots: 2.75 tiles in flight
 constexpr int kRopeSlots = 1;      // freed by its tile's QK, refilled first for the next tile
 constexpr int kPBufs = 2;          // P buffers (1 or 2): with 2 the softmax of tile i+1 need not wait for PV(i)
 static_assert(kPBufs == 1 || kPBufs == 2, "the alpha and PV-done handshakes assume at most 2");
-constexpr float kPShift = 4.0f;     // log2 of the factor carried by the softmax weights
-constexpr float kLazy = 4.75f;      // the used max moves only when exceeded by more than this
+constexpr float kPShift = 3.5f;     // log2 of the factor carried by the softmax weights
+constexpr float kLazy = 5.25f;      // the used max moves only when exceeded by more than this
+static_assert(kLazy + kPShift <= 8.8f, "p' must stay below 448, the E4M3 maximum");
 
 constexpr int kOffRing = 0;                                  // 11 pairs
 constexpr int kOffRope = kOffRing + kRingPairs * kPair;      // 180224: 2 RoPE chunks
@@ -873,7 +874,7 @@ __device__ __forceinline__ void partial_body(const DecodeArgs& args, const CUten
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
       }
-      // weights carry a 2^4 factor: p' = 2^(s - m + 4) <= 2^8.75
+      // weights carry a 2^3.5 factor: p' = 2^(s - m + 3.5) <= 2^8.75
       float pv[16];
       float psum = 0.0f;
 #pragma unroll
