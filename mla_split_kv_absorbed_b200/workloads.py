@@ -82,6 +82,10 @@ SPECS = {
     "verify_q4_256k_fp8": Spec("verify_q4_256k_fp8", B=8, q_len=4, H=64,
                                seq_lens=[262144] * 8, kv_dtype="fp8", kv_std=1.0, splits=64,
                                seed=4),
+    # profiling size: the verify shape cut to 2 requests (302 MB of KV, > L2)
+    "verify_q4_256k_b2_fp8": Spec("verify_q4_256k_b2_fp8", B=2, q_len=4, H=64,
+                                  seq_lens=[262144] * 2, kv_dtype="fp8", kv_std=1.0, splits=64,
+                                  seed=6),
 }
 
 
