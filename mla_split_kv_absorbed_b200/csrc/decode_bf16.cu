@@ -27,7 +27,9 @@
 // (warp 1), two softmax warpgroups (warps 4-11, 32 query columns each, thread
 // = token row), O^T rescale between tiles and epilogue (warps 12-15, thread =
 // latent dim).  The online softmax (log2 domain, lazy running max moving only
-// when exceeded by more than 1) and the bounded waits follow the FP8 kernel.
+// when exceeded by more than 8: bf16 weights up to 2^8 keep their 8
+// significant bits, and the O^T rescale is rarely needed; 0.4-0.8% faster
+// than a threshold of 1) and the bounded waits follow the FP8 kernel.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
                                fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
         const float m_old = sc.m_run[n];
-        const bool moved = tm > m_old + 1.0f;
+        const bool moved = tm > m_old + 8.0f;
         const float m_new = moved ? tm : m_old;
         const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
         sc.m_run[n] = m_new;
@@ -445,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; k += 2) {
           const int j = 8 * q8 + k;
-          // p = 2^(s - m) <= 2 with the lazy max; rounded to bf16 for the MMA,
+          // p = 2^(s - m) <= 2^8 with the lazy max; rounded to bf16 for the MMA,
           // and the row sum accumulates the rounded values
           const float p0 = (sv[j] == -INFINITY) ? 0.0f : ex2_approx(sv[j] - mm[k]);
           const float p1 = (sv[j + 1] == -INFINITY) ? 0.0f : ex2_approx(sv[j + 1] - mm[k + 1]);
