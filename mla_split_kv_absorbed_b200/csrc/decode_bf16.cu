@@ -409,29 +409,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j)
           if (tok >= t1 || (qq >= 0 && (int)sc.qcol[col0 + j] <= qq)) sv[j] = -INFINITY;
       }
-      float mine = -INFINITY;
+      // does any score of this group's columns exceed its used max by more
+      // than the lazy threshold?  If none does (the common case once the max
+      // has settled), the column maxima are not reduced at all.
+      bool exceed = false;
+      {
+        const float4* mo4 = reinterpret_cast<const float4*>(sc.m_run + col0);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float wm = warp_max_f32(sv[j]);
-        mine = (lane == j) ? wm : mine;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 mo = mo4[q4];
+          exceed |= sv[4 * q4] > mo.x + 8.0f;
+          exceed |= sv[4 * q4 + 1] > mo.y + 8.0f;
+          exceed |= sv[4 * q4 + 2] > mo.z + 8.0f;
+          exceed |= sv[4 * q4 + 3] > mo.w + 8.0f;
+        }
       }
-      sc.warp_max[wg][wq][lane] = mine;
       if (named_bar_or(bar_id, 128, bad || *abort_flag != 0)) {
         ok = false;
         break;
       }
-      if (wq == 0) {
-        const int n = col0 + lane;
-        const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
-                               fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
-        const float m_old = sc.m_run[n];
-        const bool moved = tm > m_old + 8.0f;
-        const float m_new = moved ? tm : m_old;
-        const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
-        sc.m_run[n] = m_new;
-        sc.alpha[i & 1][n] = a;
-        const uint32_t mask = __ballot_sync(0xffffffffu, moved);
-        if (lane == 0) sc.changed[i & 1][wg] = mask;
+      if (named_bar_or(bar_id, 128, exceed)) {
+        float mine = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float wm = warp_max_f32(sv[j]);
+          mine = (lane == j) ? wm : mine;
+        }
+        sc.warp_max[wg][wq][lane] = mine;
+        named_bar_sync(bar_id, 128);
+        if (wq == 0) {
+          const int n = col0 + lane;
+          const float tm = fmaxf(fmaxf(sc.warp_max[wg][0][lane], sc.warp_max[wg][1][lane]),
+                                 fmaxf(sc.warp_max[wg][2][lane], sc.warp_max[wg][3][lane]));
+          const float m_old = sc.m_run[n];
+          const bool moved = tm > m_old + 8.0f;
+          const float m_new = moved ? tm : m_old;
+          const float a = moved ? (m_old == -INFINITY ? 0.0f : ex2_approx(m_old - m_new)) : 1.0f;
+          sc.m_run[n] = m_new;
+          sc.alpha[i & 1][n] = a;
+          const uint32_t mask = __ballot_sync(0xffffffffu, moved);
+          if (lane == 0) sc.changed[i & 1][wg] = mask;
+        }
+      } else if (wq == 0) {
+        sc.alpha[i & 1][col0 + lane] = 1.0f;
+        if (lane == 0) sc.changed[i & 1][wg] = 0u;
       }
       named_bar_sync(bar_id, 128);
       if (wq == 0 && lane == 0) mbar_arrive(&bars[kBarAlphaFull + (i & 1)]);
